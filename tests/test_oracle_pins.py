@@ -1,0 +1,360 @@
+"""Pins for the fp64 oracle, each tied to something other than the oracle itself.
+
+Every check below comes from the Veda pages' description (sections 2.1-2.3 of
+the technical summary) plus mathematics: hand-derived examples, closed forms,
+brute force over grid coordinates, and special cases that reduce to a library
+routine (dense SDPA, logsumexp, softmax).  They are chosen so that a plausible
+mistake in the oracle -- a transposed tile order, a dropped bias or ReLU, a
+wrong scale, an off-by-one keep count, a pad slot counted as a token -- fails
+at least one of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import veda_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- helpers
+def box_members(grid, tiling):
+    """Tokens of every tile by explicit loops over box bounds (no slot formula)."""
+    T, H, W = grid
+    pt, ph, pw = tiling
+    nT, nH, nW = -(-T // pt), -(-H // ph), -(-W // pw)
+    tiles = []
+    for a in range(nT):
+        for b in range(nH):
+            for c in range(nW):
+                mem = []
+                for t in range(a * pt, min(T, (a + 1) * pt)):
+                    for y in range(b * ph, min(H, (b + 1) * ph)):
+                        for x in range(c * pw, min(W, (c + 1) * pw)):
+                            mem.append((t * H + y) * W + x)
+                tiles.append(sorted(mem))
+    return tiles
+
+
+def reshape_table(grid, tiling):
+    """Slot table by padding, reshaping and transposing an index grid."""
+    T, H, W = grid
+    pt, ph, pw = tiling
+    nT, nH, nW = -(-T // pt), -(-H // ph), -(-W // pw)
+    g = np.full((nT * pt, nH * ph, nW * pw), -1, dtype=np.int64)
+    g[:T, :H, :W] = np.arange(T * H * W).reshape(T, H, W)
+    g = g.reshape(nT, pt, nH, ph, nW, pw).transpose(0, 2, 4, 1, 3, 5)
+    return g.reshape(-1)
+
+
+def read_golden_tables():
+    cases = []
+    with open(os.path.join(GOLDEN, "permutation_examples.txt")) as f:
+        lines = [ln.strip() for ln in f if ln.strip() and not ln.startswith("#")]
+    for hdr, body in zip(lines[0::2], lines[1::2]):
+        p = hdr.split()
+        grid = (int(p[1]), int(p[2]), int(p[3]))
+        tiling = (int(p[5]), int(p[6]), int(p[7]))
+        table = [int(v) for v in body.replace("|", " ").split()]
+        cases.append((grid, tiling, np.array(table)))
+    return cases
+
+
+GRIDS = [((4, 8, 8), (1, 8, 8)), ((4, 8, 8), (4, 4, 4)), ((3, 5, 7), (1, 2, 4)),
+         ((3, 5, 7), (2, 2, 2)), ((5, 9, 6), (2, 4, 2)), ((2, 3, 17), (1, 1, 16))]
+
+
+# ---------------------------------------------------------------- step 1: tiling
+def test_slot_table_hand_examples():
+    cases = read_golden_tables()
+    assert len(cases) == 4
+    for grid, tiling, table in cases:
+        np.testing.assert_array_equal(O.slot_table(grid, tiling), table)
+
+
+@pytest.mark.parametrize("grid,tiling", GRIDS)
+def test_slot_table_matches_reshape_construction(grid, tiling):
+    np.testing.assert_array_equal(O.slot_table(grid, tiling), reshape_table(grid, tiling))
+
+
+@pytest.mark.parametrize("grid,tiling", GRIDS)
+def test_tile_membership_matches_box_bounds(grid, tiling):
+    S = tiling[0] * tiling[1] * tiling[2]
+    tab = O.slot_table(grid, tiling)
+    mem = box_members(grid, tiling)
+    assert tab.size == len(mem) * S
+    for j, m in enumerate(mem):
+        got = sorted(int(v) for v in tab[j * S:(j + 1) * S] if v >= 0)
+        assert got == m
+
+
+def test_frame_tiling_is_identity():
+    # A (1,8,8) tile over an 8x8 frame holds exactly one frame in raster order.
+    np.testing.assert_array_equal(O.slot_table((4, 8, 8), (1, 8, 8)), np.arange(256))
+
+
+@pytest.mark.parametrize("grid,tiling", GRIDS)
+def test_permute_unpermute_identity_and_zero_pads(grid, tiling):
+    rng = np.random.default_rng(0)
+    S = tiling[0] * tiling[1] * tiling[2]
+    other = (tiling[2], tiling[1], tiling[0])          # second head, another tiling of the same size
+    tilings = [tiling, other]
+    N = grid[0] * grid[1] * grid[2]
+    x = rng.standard_normal((2, 2, N, 8))
+    xp = O.tile_permute(x, grid, tilings, S)
+    np.testing.assert_array_equal(O.tile_unpermute(xp, grid, tilings, S), x)
+    for h, tl in enumerate(tilings):
+        tab = O.slot_table(grid, tl)
+        full = np.full(xp.shape[2], -1)
+        full[:tab.size] = tab
+        assert np.all(xp[:, h, full < 0] == 0)
+        # every grid token appears exactly once
+        assert sorted(tab[tab >= 0].tolist()) == list(range(N))
+
+
+def test_tile_counts_configs():
+    # Tile counts quoted for the workloads (hand arithmetic: ceil per dim).
+    assert O.num_tiles((21, 30, 52), (2, 8, 8)) == 11 * 4 * 7 == 308
+    assert O.num_tiles((21, 30, 52), (1, 8, 16)) == 21 * 4 * 4 == 336
+    assert O.num_tiles((21, 45, 80), (8, 4, 4)) == 3 * 12 * 20 == 720
+    assert O.num_tiles((60, 64, 64), (2, 8, 8)) == 30 * 8 * 8 == 1920
+
+
+# ---------------------------------------------------------------- step 2: TripPool
+def test_tripool_closed_forms():
+    grid, tiling, S = (1, 3, 3), (1, 2, 2), 4
+    d = 3
+    x = np.zeros((1, 1, 9, d))
+    # channel 0: constant 2.5; channel 1: token index; channel 2: -index
+    x[0, 0, :, 0] = 2.5
+    x[0, 0, :, 1] = np.arange(9)
+    x[0, 0, :, 2] = -np.arange(9)
+    desc = O.tripool(O.tile_permute(x, grid, [tiling], S), grid, [tiling], S)[0, 0]
+    # tile 0 = tokens {0,1,3,4}; tile 1 = {2,5}; tile 2 = {6,7}; tile 3 = {8}
+    members = [[0, 1, 3, 4], [2, 5], [6, 7], [8]]
+    for j, m in enumerate(members):
+        mean, mx, mn = desc[j, :d], desc[j, d:2 * d], desc[j, 2 * d:]
+        assert mean[0] == mx[0] == mn[0] == 2.5
+        assert mean[1] == pytest.approx(sum(m) / len(m))
+        assert mx[1] == max(m) and mn[1] == min(m)
+        assert mx[2] == -min(m) and mn[2] == -max(m)
+
+
+@pytest.mark.parametrize("grid,tiling", GRIDS)
+def test_tripool_brute_force_over_grid(grid, tiling):
+    rng = np.random.default_rng(1)
+    S = tiling[0] * tiling[1] * tiling[2]
+    N = grid[0] * grid[1] * grid[2]
+    x = rng.standard_normal((1, 1, N, 5))
+    desc = O.tripool(O.tile_permute(x, grid, [tiling], S), grid, [tiling], S)[0, 0]
+    for j, m in enumerate(box_members(grid, tiling)):
+        rows = torch.tensor(x[0, 0, m])
+        ref = torch.cat([rows.mean(0), rows.amax(0), rows.amin(0)]).numpy()
+        np.testing.assert_allclose(desc[j], ref, rtol=1e-14, atol=1e-14)
+        assert np.all(desc[j, 5:10] >= desc[j, :5]) and np.all(desc[j, :5] >= desc[j, 10:])
+
+
+# ---------------------------------------------------------------- step 3: estimator
+def test_estimator_bias_only_closed_form():
+    # W1 = 0, b1 = c > 0 -> hidden = c (ReLU passes) -> phi = c * W2 @ 1 + b2.
+    rng = np.random.default_rng(2)
+    desc = rng.standard_normal((4, 6))
+    w1 = np.zeros((5, 6)); b1 = np.full(5, 0.7)
+    w2 = rng.standard_normal((3, 5)); b2 = np.array([0.1, -0.2, 0.3])
+    phi = O.estimator_head(desc, w1, b1, w2, b2)
+    expect = 0.7 * w2.sum(axis=1) + b2
+    for r in range(4):
+        np.testing.assert_allclose(phi[r], expect, rtol=1e-14)
+
+
+def test_estimator_relu_closed_form():
+    # W1 = [I; -I] over the mean block: hidden = (relu(m), relu(-m)), W2 = [I, -I] -> phi = m.
+    d = 4
+    desc = np.array([[0.5, -1.0, 2.0, -0.25] + [9.0] * 8])
+    w1 = np.zeros((2 * d, 3 * d)); w1[:d, :d] = np.eye(d); w1[d:, :d] = -np.eye(d)
+    w2 = np.hstack([np.eye(d), -np.eye(d)])
+    phi = O.estimator_head(desc, w1, np.zeros(2 * d), w2, np.zeros(d))
+    np.testing.assert_allclose(phi[0], desc[0, :d], rtol=0, atol=0)
+    # Dropping the second half of hidden (only relu(m)) must not reproduce m.
+    phi_pos = O.estimator_head(desc, w1[:d], np.zeros(d), np.eye(d), np.zeros(d))
+    np.testing.assert_allclose(phi_pos[0], np.maximum(desc[0, :d], 0))
+
+
+def test_scores_scale_and_orientation():
+    # phi_q rows = e_0 * a_i, phi_k rows = e_0 * b_j  ->  s[i,j] = a_i * b_j / sqrt(e).
+    e, d3 = 16, 6
+    a = np.array([1.0, 2.0, -1.0]); bvals = np.array([3.0, -0.5])
+    desc_q = np.zeros((3, d3)); desc_q[:, 0] = a
+    desc_k = np.zeros((2, d3)); desc_k[:, 0] = bvals
+    w1 = np.zeros((2, d3)); w1[0, 0] = 1; w1[1, 0] = -1
+    w2 = np.zeros((e, 2)); w2[0, 0] = 1; w2[0, 1] = -1
+    wts = (w1, np.zeros(2), w2, np.zeros(e))
+    s = O.tile_scores_head(desc_q, desc_k, wts, wts)
+    np.testing.assert_allclose(s, np.outer(a, bvals) / 4.0, rtol=1e-15)
+
+
+def test_row_softmax_matches_scipy():
+    from scipy.special import softmax
+    rng = np.random.default_rng(3)
+    s = rng.standard_normal((7, 11)) * 5
+    np.testing.assert_allclose(O.row_softmax(s), softmax(s, axis=1), rtol=1e-13)
+    np.testing.assert_allclose(O.row_softmax(s).sum(1), 1.0, rtol=1e-14)
+
+
+# ---------------------------------------------------------------- step 4: top-k
+def test_keep_count_table():
+    assert O.keep_count(4, 0.5) == 2
+    assert [O.keep_count(n, 0.1) for n in (308, 336, 312)] == [31, 34, 31]
+    assert [O.keep_count(n, 0.05) for n in (660, 630, 720)] == [33, 32, 36]
+    assert [O.keep_count(n, 0.05) for n in (512, 960, 1920)] == [26, 48, 96]
+    assert O.keep_count(10, 1e-6) == 1 and O.keep_count(10, 1.0) == 10
+
+
+def test_topk_against_python_sort_with_ties():
+    rng = np.random.default_rng(4)
+    for trial in range(50):
+        nt = int(rng.integers(1, 80))
+        s = np.round(rng.standard_normal(nt), 1)         # many exact ties
+        k = int(rng.integers(1, nt + 1))
+        ref = sorted(sorted(range(nt), key=lambda j: (-s[j], j))[:k])
+        assert O.select_topk_row(s, k).tolist() == ref
+    s = rng.standard_normal(13)
+    assert O.select_topk_row(s, 13).tolist() == list(range(13))
+
+
+def test_score_topk_contract():
+    grid, tilings, S = (3, 5, 7), [(1, 2, 4), (2, 2, 2)], 8
+    rng = np.random.default_rng(5)
+    nts, ntmax = O.tile_layout(grid, tilings)
+    dq = rng.standard_normal((1, 2, ntmax, 12)); dk = rng.standard_normal((1, 2, ntmax, 12))
+    mlp = (rng.standard_normal((2, 6, 12)), rng.standard_normal((2, 6)),
+           rng.standard_normal((2, 5, 6)), rng.standard_normal((2, 5)))
+    idx, probs = O.score_topk(dq, dk, grid, tilings, S, mlp, mlp, 0.3)
+    for h, nt in enumerate(nts):
+        k = O.keep_count(nt, 0.3)
+        for i in range(ntmax):
+            row = idx[0, h, i]
+            if i >= nt:
+                assert np.all(row == -1)
+                continue
+            sel = row[row >= 0]
+            assert len(sel) == k and np.all(np.diff(sel) > 0) and sel.max() < nt
+            assert np.all(row[k:] == -1)
+            np.testing.assert_allclose(probs[0, h, i, :nt].sum(), 1.0, rtol=1e-13)
+
+
+# ---------------------------------------------------------------- step 5: attention
+def _inputs(grid, d, heads=2, seed=6):
+    rng = np.random.default_rng(seed)
+    N = grid[0] * grid[1] * grid[2]
+    return [rng.standard_normal((1, heads, N, d)) for _ in range(3)]
+
+
+def _dense_sdpa(q, k, v):
+    tq, tk, tv = (torch.tensor(a) for a in (q, k, v))
+    return torch.nn.functional.scaled_dot_product_attention(tq, tk, tv).numpy()
+
+
+@pytest.mark.parametrize("grid,tilings,S", [((4, 8, 8), [(1, 8, 8), (4, 4, 4)], 64),
+                                             ((3, 5, 7), [(1, 2, 4), (2, 2, 2)], 8)])
+def test_full_keep_equals_dense_sdpa(grid, tilings, S):
+    q, k, v = _inputs(grid, 16)
+    qp, kp, vp = (O.tile_permute(a, grid, tilings, S) for a in (q, k, v))
+    nts, ntmax = O.tile_layout(grid, tilings)
+    idx = np.full((1, 2, ntmax, ntmax), -1, dtype=np.int32)
+    for h, nt in enumerate(nts):
+        idx[0, h, :nt, :nt] = np.arange(nt)
+    op, lse = O.sparse_attention(qp, kp, vp, idx, grid, tilings, S)
+    o = O.tile_unpermute(op, grid, tilings, S)
+    np.testing.assert_allclose(o, _dense_sdpa(q, k, v), rtol=1e-12, atol=1e-12)
+    ref_lse = torch.logsumexp(torch.tensor(q) @ torch.tensor(k).transpose(-1, -2) / 4.0, dim=-1).numpy()
+    lse_grid = O.tile_unpermute(lse[..., None], grid, tilings, S)[..., 0]
+    np.testing.assert_allclose(lse_grid, ref_lse, rtol=1e-12, atol=1e-12)
+
+
+def test_masked_attention_brute_force_in_grid_coordinates():
+    grid, tilings, S = (3, 5, 7), [(1, 2, 4), (2, 2, 2)], 8
+    q, k, v = _inputs(grid, 8, seed=7)
+    rng = np.random.default_rng(8)
+    nts, ntmax = O.tile_layout(grid, tilings)
+    idx = np.full((1, 2, ntmax, 4), -1, dtype=np.int32)
+    for h, nt in enumerate(nts):
+        for i in range(nt):
+            idx[0, h, i, :3] = np.sort(rng.choice(nt, 3, replace=False))
+    qp, kp, vp = (O.tile_permute(a, grid, tilings, S) for a in (q, k, v))
+    op, _ = O.sparse_attention(qp, kp, vp, idx, grid, tilings, S)
+    o = O.tile_unpermute(op, grid, tilings, S)
+    N = grid[0] * grid[1] * grid[2]
+    for h in range(2):
+        members = box_members(grid, tilings[h])
+        tile_of = np.empty(N, dtype=np.int64)
+        for j, m in enumerate(members):
+            tile_of[m] = j
+        allowed = np.zeros((N, N), dtype=bool)
+        for n in range(N):
+            sel = set(int(j) for j in idx[0, h, tile_of[n]] if j >= 0)
+            allowed[n] = [tile_of[m] in sel for m in range(N)]
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.tensor(q[0, h]), torch.tensor(k[0, h]), torch.tensor(v[0, h]),
+            attn_mask=torch.tensor(allowed)).numpy()
+        np.testing.assert_allclose(o[0, h], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_tiling_invariance_at_full_keep():
+    grid, S = (4, 8, 8), 64
+    q, k, v = _inputs(grid, 8, heads=1, seed=9)
+    outs = []
+    for tl in [(1, 8, 8), (4, 4, 4), (2, 4, 8), (4, 2, 8)]:
+        qp, kp, vp = (O.tile_permute(a, grid, [tl], S) for a in (q, k, v))
+        nt = O.num_tiles(grid, tl)
+        idx = np.tile(np.arange(nt, dtype=np.int32), (1, 1, nt, 1))
+        op, _ = O.sparse_attention(qp, kp, vp, idx, grid, [tl], S)
+        outs.append(O.tile_unpermute(op, grid, [tl], S))
+    for o in outs[1:]:
+        np.testing.assert_allclose(o, outs[0], rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- secondary: tile map
+@pytest.mark.parametrize("grid,tiling", [((4, 8, 8), (4, 4, 4)), ((3, 5, 7), (2, 2, 2))])
+def test_tile_map_equals_maxpool_of_explicit_softmax(grid, tiling):
+    S = tiling[0] * tiling[1] * tiling[2]
+    q, k, _ = _inputs(grid, 8, heads=1, seed=10)
+    qp, kp = (O.tile_permute(a, grid, [tiling], S) for a in (q, k))
+    nt = O.num_tiles(grid, tiling)
+    rows = np.array([[i for i in range(nt)]], dtype=np.int32)
+    M = O.tile_map_maxpool(qp, kp, rows, grid, [tiling], S)[0, 0]
+    P = torch.softmax(torch.tensor(q[0, 0]) @ torch.tensor(k[0, 0]).T / math.sqrt(8), dim=-1).numpy()
+    members = box_members(grid, tiling)
+    N = P.shape[0]
+    for i, mi in enumerate(members):
+        for j, mj in enumerate(members):
+            assert M[i, j] == pytest.approx(P[np.ix_(mi, mj)].max(), rel=1e-12)
+        assert M[i].max() >= 1.0 / N
+    assert np.all(M > 0) and np.all(M <= 1)
+
+
+def test_tile_map_unused_rows_zero():
+    grid, tiling, S = (3, 5, 7), (2, 2, 2), 8
+    q, k, _ = _inputs(grid, 4, heads=1, seed=11)
+    qp, kp = (O.tile_permute(a, grid, [tiling], S) for a in (q, k))
+    rows = np.array([[2, -1, 0]], dtype=np.int32)
+    M = O.tile_map_maxpool(qp, kp, rows, grid, [tiling], S)[0, 0]
+    assert np.all(M[1] == 0) and np.all(M[0] > 0) and np.all(M[2] > 0)
+
+
+# ---------------------------------------------------------------- whole path
+def test_forward_tiny_shapes_and_full_keep_reduction():
+    from veda_synth import PRESETS, make_qkv, make_mlp
+    w = PRESETS["tiny"]
+    q, k, v = (t.to(torch.float64).numpy() for t in make_qkv(w, seed=0))
+    m = make_mlp(w, seed=1)
+    mlp = tuple(t.numpy() for t in (m.w1, m.b1, m.w2, m.b2))
+    grid = (w.T, w.H, w.W)
+    out = O.forward(q, k, v, grid, w.tilings, w.S, mlp, mlp, 1.0)
+    np.testing.assert_allclose(out["o"], _dense_sdpa(q, k, v), rtol=1e-12, atol=1e-12)
+    out = O.forward(q, k, v, grid, w.tilings, w.S, mlp, mlp, w.keep)
+    assert out["idx"].shape == (1, 2, 4, 2)
+    assert np.all(out["idx"] >= 0)
