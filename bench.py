@@ -1,0 +1,349 @@
+#!/usr/bin/env python3
+"""Benchmark of the tile-sparse attention layer (Veda, head-aware tiles) on B200.
+
+One step = one attention layer of the inference path on one GPU:
+    permute Q, K, V -> TripPool Q, K -> estimator + softmax + top-k
+    -> tile-skipping attention -> unpermute,
+all through the C ABI, inputs resident in HBM.  Default workload: the
+Wan2.1-14B 720p/81-frame shape (21x45x80 grid = 75,600 tokens, 40 heads,
+d = 128, 128-token per-head tiles, keep 5% = 95% sparsity).
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the fp64 CPU
+oracle on a bounded sample of the same workload instead.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own layer
+(a different seed) with no data-path collective -- the heads of a layer are
+independent, so the work partitions -- and the reported time is the max over
+ranks (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "tile-sparse attn ms/layer & kept-tile TFLOP/s (% of B200 BF16 peak) at 95% sparsity"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+WORKLOAD_NAMES = {"wan14b": "Wan2.1-14B-720p-81f 21x45x80 (75,600 tokens) 40 heads d128 keep 5%",
+                  "wan14b-k10": "Wan2.1-14B-720p-81f 21x45x80 40 heads d128 keep 10%",
+                  "wan14b-dense": "Wan2.1-14B-720p-81f 21x45x80 40 heads d128 keep 100% (dense reference)",
+                  "wan1.3b": "Wan2.1-1.3B-480p 21x30x52 (32,760 tokens) 12 heads d128 keep 10%",
+                  "long": "long video 31x45x80 (111,600 tokens) 24 heads d128 keep 5%",
+                  "sweep61k": "sweep 15x64x64 (61,440 tokens) 24 heads (2,8,8) keep 5%",
+                  "sweep123k": "sweep 30x64x64 (122,880 tokens) 24 heads (2,8,8) keep 5%",
+                  "sweep246k": "sweep 60x64x64 (245,760 tokens) 24 heads (2,8,8) keep 5%",
+                  "tiny": "tiny 4x8x8 2 heads d64"}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kept_flops(nts, ks, B, S, d):
+    """Algorithmic FLOPs of the tile-skipping attention: 4*S^2*d per kept (Q tile, K tile) pair."""
+    return float(B * sum(nt * k for nt, k in zip(nts, ks)) * 4 * S * S * d)
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [ln.strip().split(",") for ln in self.file.read().splitlines() if ln.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = max(mx, float(r[2]))
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args, world, rank, local):
+    import tile_sparse_attention_head_b200 as V
+    from veda_synth import PRESETS, make_mlp, make_qkv
+
+    w = PRESETS[args.workload]
+    p = V.Problem(w.B, w.heads, w.d, w.S, (w.T, w.H, w.W), w.tilings)
+    q, k, v = make_qkv(w, seed=rank)
+    m = make_mlp(w, seed=1)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    mlp = tuple(t.to(dev) for t in (m.w1, m.b1, m.w2, m.b2))
+    att = V.VedaAttention(p, mlp, mlp, w.keep, device=dev)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    out = torch.empty(p.grid_shape(), dtype=torch.bfloat16, device=dev)
+    ks, _ = p.keep_count(w.keep)
+    flops = kept_flops(p.nt_per_head, ks, w.B, w.S, w.d)
+    stream = torch.cuda.current_stream()
+
+    # per-stage events for one instrumented step (after warm-up)
+    def step(ev=None):
+        if ev is None:
+            att(qd, kd, vd, out)
+            return
+        ev[0].record()
+        V.veda_tile_permute(p, qd, att.qp)
+        V.veda_tile_permute(p, kd, att.kp)
+        V.veda_tile_permute(p, vd, att.vp)
+        ev[1].record()
+        V.veda_tripool(p, att.qp, att.desc_q)
+        V.veda_tripool(p, att.kp, att.desc_k)
+        ev[2].record()
+        V.veda_tile_score_topk(p, att.desc_q, att.desc_k, att.mlp_q, att.mlp_k, att.keep, att.idx, None,
+                               att.workspace)
+        ev[3].record()
+        V.veda_tile_sparse_attn(p, att.qp, att.kp, att.vp, att.idx, att.op)
+        ev[4].record()
+        V.veda_tile_unpermute(p, att.op, out)
+        ev[5].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    V.veda_sync_status()
+
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    V.veda_sync_status()
+    ms_total = max_over_ranks(t0.elapsed_time(t1), world)
+    ms_step = ms_total / args.steps
+    stage = {"permute": [], "tripool": [], "score_topk": [], "attention": [], "unpermute": []}
+    for ev in evs:
+        for name, a, b in (("permute", 0, 1), ("tripool", 1, 2), ("score_topk", 2, 3), ("attention", 3, 4),
+                           ("unpermute", 4, 5)):
+            stage[name].append(ev[a].elapsed_time(ev[b]))
+    stage_ms = {k: float(np.mean(v)) for k, v in stage.items()}
+    attn_ms = max_over_ranks(stage_ms["attention"], world)
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+        oh = torch.empty(p.grid_shape(), dtype=torch.bfloat16).pin_memory()
+        for _ in range(2):
+            qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
+            att(qd, kd, vd, out)
+            oh.copy_(out, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        n_e2e = max(3, args.steps // 4)
+        for _ in range(n_e2e):
+            qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
+            att(qd, kd, vd, out)
+            oh.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
+        nbytes = lambda t: t.numel() * t.element_size()
+        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": nbytes(q) + nbytes(k) + nbytes(v), "d2h_bytes_per_step": nbytes(oh),
+               "steps": n_e2e}
+
+    peaks, peak_src = load_peaks()
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "kernel": "sparse_attn_kernel<128,128>", "peak_source": f"{peak_src} bf16 burst",
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]}
+    res = {"metric": METRIC, "value": world * flops / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+           "config": {"workload": WORKLOAD_NAMES.get(args.workload, args.workload), "preset": args.workload,
+                      "grid": [w.T, w.H, w.W], "tokens": w.N, "heads": w.heads, "d": w.d, "S": w.S,
+                      "keep": w.keep, "tilings": "per head from {(2,8,8),(1,8,16),(8,4,4),(4,4,8)}",
+                      "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"replicas x{world}",
+                      "kept_tile_flops_per_layer": flops,
+                      "l2": "inputs (3 x %.0f MB) larger than L2; no flush" % (q.numel() * 2 / 1e6)},
+           "ms_per_layer": ms_step, "stage_ms": stage_ms, "attn_tflops": achieved,
+           "pct_of_bf16_peak": 100.0 * achieved / peaks["bf16_tflops"],
+           "roofline": roofline, "gpu_launches": 9 * args.steps, "clocks": clk, "e2e": e2e}
+    return res, (w, p, ks, flops)
+
+
+def cpu_sample_oracle(w, p_nts, ks, heads=1, tiles=None, seed=0):
+    """Oracle over a bounded sample: `heads` heads, full permute/pool/score/top-k, attention for
+    `tiles` Q tiles per head (all if None).  Returns (seconds, kept FLOPs processed, description)."""
+    from oracle import veda_oracle as O
+    from veda_synth import make_mlp, make_qkv
+    q, k, v = make_qkv(w, seed=seed, heads=heads)
+    m = make_mlp(w, seed=1, heads=heads)
+    mlp = tuple(t.numpy().astype(np.float64) for t in (m.w1, m.b1, m.w2, m.b2))
+    grid = (w.T, w.H, w.W)
+    tl = list(w.tilings[:heads])
+    qd, kd, vd = (t.to(torch.float64).numpy() for t in (q, k, v))
+    t0 = time.perf_counter()
+    qp, kp, vp = (O.tile_permute(a, grid, tl, w.S) for a in (qd, kd, vd))
+    dq, dk = O.tripool(qp, grid, tl, w.S), O.tripool(kp, grid, tl, w.S)
+    idx, _ = O.score_topk(dq, dk, grid, tl, w.S, mlp, mlp, float(np.float32(w.keep)))
+    done = 0.0
+    scale = 1 / math.sqrt(w.d)
+    for h in range(heads):
+        tab = O.slot_table(grid, tl[h])
+        nt = p_nts[h]
+        sel = range(nt) if tiles is None else range(min(tiles, nt))
+        for i in sel:
+            O.attention_tile(qp[0, h], kp[0, h], vp[0, h], tab, i, idx[0, h, i], w.S, scale)
+            done += ks[h] * 4 * w.S * w.S * w.d
+    secs = time.perf_counter() - t0
+    desc = (f"{heads} head(s) of {w.name}: full permute+TripPool+score/top-k, attention for "
+            f"{'all' if tiles is None else tiles} Q tiles per head")
+    return secs, done, desc
+
+
+def run_reference(args, world, rank):
+    """The fp64 CPU oracle as the reference arm, timed on the host cores."""
+    from veda_synth import PRESETS
+    from oracle import veda_oracle as O
+    w = PRESETS[args.workload]
+    nts, _ = O.tile_layout((w.T, w.H, w.W), w.tilings)
+    ks = [O.keep_count(n, float(np.float32(w.keep))) for n in nts]
+    tiles = args.ref_tiles
+    for _ in range(args.warmup):
+        cpu_sample_oracle(w, nts, ks, heads=1, tiles=max(1, tiles // 8))
+    secs, flops = 0.0, 0.0
+    desc = ""
+    for s in range(args.steps):
+        t, f, desc = cpu_sample_oracle(w, nts, ks, heads=1, tiles=tiles, seed=s)
+        secs += t
+        flops += f
+    value = flops / secs / 1e12
+    cores = os.cpu_count()
+    return {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD_NAMES.get(args.workload, args.workload), "preset": args.workload,
+                       "parallelism": "cpu"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="wan14b")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-tiles", type=int, default=24, help="Q tiles per oracle sample (reference arm)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args, world, rank)), flush=True)
+        return
+
+    world, rank, local = dist_setup(args.gpus)
+    res, (w, p, ks, flops) = run_ours(args, world, rank, local)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            secs, done, desc = cpu_sample_oracle(w, p.nt_per_head, ks, heads=1, tiles=96)
+            res["cpu_baseline"] = {"value": done / secs / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
+                                   "kind": "oracle", "sample": desc, "seconds": secs}
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

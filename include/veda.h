@@ -1,0 +1,215 @@
+/*
+ * veda.h -- C ABI of the B200 (sm_100a) tile-sparse attention library.
+ *
+ * The method is Veda's head-aware tile-sparse self-attention over a T x H x W
+ * video token grid ("Veda: Scalable Video Diffusion via Distilled Sparse
+ * Attention", technical summary, sections 2.1-2.3).  The inference path is
+ *
+ *   veda_tile_permute (Q, K, V)  ->  veda_tripool (Q, K)  ->  veda_tile_score_topk
+ *   ->  veda_tile_sparse_attn  ->  veda_tile_unpermute
+ *
+ * and the distillation target is built by veda_tile_map_maxpool.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Layout.  Grid-order tensors are [B, heads, N, d] row-major bf16 with
+ *   N = T*H*W and grid index n = (t*H + y)*W + x.  Tile-major ("permuted")
+ *   tensors are [B, heads, NT_max*S, d] bf16: head h's tile j occupies rows
+ *   j*S .. j*S+S-1, S = pt*ph*pw, and NT_max is the largest tile count over
+ *   heads (veda_tile_layout).  Inside a tile, slots are row-major over
+ *   (t, y, x) offsets; tiles are row-major over tile coordinates; a grid
+ *   dimension that its factor does not divide is padded up to a multiple of
+ *   it.  Pad slots hold no token.
+ * Memory.  Every tensor pointer is caller-owned DEVICE memory, 16-byte
+ *   aligned, and must not alias another argument of the same call unless the
+ *   call says so.  The library allocates no device memory; calls that need
+ *   scratch take a caller-provided workspace whose size a *_workspace query
+ *   returns.
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  Every call only enqueues work and returns; nothing synchronises.
+ *   Faults and kernel time-outs surface through veda_sync_status().
+ * Errors.  Every call validates its arguments on the host first and returns
+ *   VEDA_ERR_INVALID_ARG / VEDA_ERR_UNSUPPORTED without launching anything;
+ *   veda_last_error() returns a thread-local description of the last failure.
+ * Sizes.  d in {64, 128}; S in {64, 128} with pt*ph*pw == S for every head;
+ *   1 <= heads <= VEDA_MAX_HEADS; B >= 1; every grid dimension >= 1.
+ */
+#ifndef VEDA_H_
+#define VEDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VEDA_MAX_HEADS 128
+
+typedef enum {
+  VEDA_OK = 0,
+  VEDA_ERR_INVALID_ARG = 1,   /* bad pointer, size, ratio or tiling */
+  VEDA_ERR_UNSUPPORTED = 2,   /* valid request outside the built shapes (d, S) */
+  VEDA_ERR_CUDA = 3,          /* a CUDA runtime call or a launch failed */
+  VEDA_ERR_TIMEOUT = 4        /* a kernel gave up on a bounded wait (device error word set) */
+} veda_status;
+
+/* Video token grid: frames T, height H, width W (latent tokens). */
+typedef struct { int32_t T, H, W; } veda_grid;
+
+/* One head's tile factorisation pi = (p_t, p_h, p_w) of the tile size S
+ * ("Head-aware tiling", section 2.2: each layer and head factorises the
+ * hardware tile size in its own way). */
+typedef struct { int32_t pt, ph, pw; } veda_tiling;
+
+/* Problem statement shared by all calls.  `tilings` is a HOST array of
+ * `heads` entries, read during the call only. */
+typedef struct {
+  int32_t B, heads, d, S;
+  veda_grid grid;
+  const veda_tiling* tilings;
+} veda_problem;
+
+/* Per-head two-layer estimator (section 2.1, "head-specific MLP
+ * projections"): phi = W2 relu(W1 desc + b1) + b2.  DEVICE fp32 pointers:
+ * w1 [heads, hidden, 3d], b1 [heads, hidden], w2 [heads, e, hidden],
+ * b2 [heads, e], all row-major.  hidden <= 512, e <= 128, e % 4 == 0. */
+typedef struct {
+  const float* w1;
+  const float* b1;
+  const float* w2;
+  const float* b2;
+  int32_t hidden, e;
+} veda_mlp;
+
+/* ---------------------------------------------------------------- host helpers */
+
+/* Tiles per head after padding, NT_h = ceil(T/pt)*ceil(H/ph)*ceil(W/pw), and
+ * their maximum.  `nt_per_head` is a HOST array of `heads` entries (may be
+ * NULL); `nt_max` a host scalar (may be NULL).  Pure host arithmetic. */
+veda_status veda_tile_layout(const veda_problem* p, int32_t* nt_per_head, int32_t* nt_max);
+
+/* Kept K tiles per Q tile for keep ratio r in (0, 1]:
+ * k_h = max(1, min(NT_h, floor(r*NT_h + 1/2))) (the pages fix only "keep
+ * about 5-10% of tiles"; this rounding is this library's reading).  Host
+ * arrays as in veda_tile_layout. */
+veda_status veda_keep_count(const veda_problem* p, float keep_ratio, int32_t* k_per_head,
+                            int32_t* k_max);
+
+/* ---------------------------------------------------------------- step 1: tiling */
+
+/* Per-head token permutation, grid order -> tile-major (section 2.2).
+ * x  [B, heads, N, d] bf16 (read), xp [B, heads, NT_max*S, d] bf16 (written
+ * in full: pad slots and rows of tiles j >= NT_h are written as zeros).
+ * x and xp must not overlap. */
+veda_status veda_tile_permute(const veda_problem* p, const void* x, void* xp, void* stream);
+
+/* Inverse of veda_tile_permute on token rows ("output scattered back to grid
+ * order"): xp [B, heads, NT_max*S, d] bf16 (read), x [B, heads, N, d] bf16
+ * (every row written).  Pad rows of xp are ignored. */
+veda_status veda_tile_unpermute(const veda_problem* p, const void* xp, void* x, void* stream);
+
+/* ---------------------------------------------------------------- step 2: TripPool */
+
+/* TripPool descriptor per tile (section 2.1, "statistics-aware estimator":
+ * channel-wise mean, max and min concatenated).  xp [B, heads, NT_max*S, d]
+ * bf16 tile-major (read); desc [B, heads, NT_max, 3d] fp32 (written in full):
+ * desc[.., j, 0:d] = mean, [d:2d] = max, [2d:3d] = min over the token slots of
+ * tile j (pad slots excluded); rows j >= NT_h are zero. */
+veda_status veda_tripool(const veda_problem* p, const void* xp, float* desc, void* stream);
+
+/* ---------------------------------------------------------------- steps 3-4: estimator + top-k */
+
+/* Bytes of workspace veda_tile_score_topk needs for estimator width e. */
+veda_status veda_score_topk_workspace(const veda_problem* p, int32_t e, size_t* bytes);
+
+/* Distilled tile scoring and selection (section 2.1 "distilled tile scoring",
+ * "row-wise distribution over tiles"; news page "95% sparsity").
+ * desc_q, desc_k [B, heads, NT_max, 3d] fp32 (read).  mlp_q / mlp_k: HOST
+ * structs holding device weight pointers; they may describe the same
+ * weights.  For each head and valid Q tile i:
+ *   s[i, j] = <phi_q(desc_q[i]), phi_k(desc_k[j])> / sqrt(e),  j < NT_h,
+ *   probs[i, :] = softmax_j s[i, :]                (optional),
+ *   idx[i, :] = the k_h indices j of largest s[i, j], ties to the smaller j,
+ *               ascending, then -1 up to k_max.
+ * idx [B, heads, NT_max, k_max] int32 (written in full; rows i >= NT_h are -1);
+ * k_max >= max_h k_h (veda_keep_count).  probs [B, heads, NT_max, NT_max]
+ * fp32 or NULL (written in full, zero outside the valid block).
+ * workspace: device scratch of >= veda_score_topk_workspace() bytes, 256-byte
+ * aligned, owned by the caller, not read before it is written. */
+veda_status veda_tile_score_topk(const veda_problem* p, const float* desc_q, const float* desc_k,
+                                 const veda_mlp* mlp_q, const veda_mlp* mlp_k, float keep_ratio,
+                                 int32_t* idx, int32_t k_max, float* probs, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------- step 5: tile-skipping attention */
+
+/* Block-sparse attention over only the selected K/V tiles (section 2.3,
+ * "tile-skipping sparse attention kernel"; news page "tile skipping").
+ * qp, kp, vp [B, heads, NT_max*S, d] bf16 tile-major (read).
+ * idx [B, heads, NT_max, k_max] int32: per Q tile the selected K tiles, each
+ * in [0, NT_h), distinct, terminated by -1 or by k_max entries; at least one
+ * entry per valid Q tile.  For every token slot q of Q tile i:
+ *   op[q] = sum_key softmax(scale * <Q_q, K_key>) V_key over the token slots of
+ *   the selected tiles (pad key slots masked),
+ *   lse[q] = ln sum_key exp(scale * <Q_q, K_key>).
+ * scale <= 0 selects 1/sqrt(d).  op [B, heads, NT_max*S, d] bf16: token rows
+ * written, pad rows and rows of tiles i >= NT_h left unspecified.  lse
+ * [B, heads, NT_max*S] fp32 or NULL, same row rule.  Runs on the tcgen05
+ * tensor cores; fp32 accumulation. */
+veda_status veda_tile_sparse_attn(const veda_problem* p, const void* qp, const void* kp,
+                                  const void* vp, const int32_t* idx, int32_t k_max, float scale,
+                                  void* op, float* lse, void* stream);
+
+/* ---------------------------------------------------------------- secondary: tile map */
+
+/* Bytes of workspace veda_tile_map_maxpool needs for R subset rows. */
+veda_status veda_tile_map_workspace(const veda_problem* p, int32_t R, size_t* bytes);
+
+/* Max-pooled full-attention tile map, the distillation target (section 2.1
+ * "target construction": max-pool the full attention matrix over Q-tile x
+ * K-tile regions; section 2.3: built in two passes over a random subset of Q
+ * tiles).  qp, kp [B, heads, NT_max*S, d] bf16 tile-major (read).
+ * rows [B*heads, R] int32: Q tiles of the subset per (b, h), each in
+ * [0, NT_h) or -1 (unused).  With P the softmax of scale * Q K^T over every
+ * valid key of the head:
+ *   map[b, h, r, j] = max_{q in tile rows[r], key in tile j} P[q, key]
+ * for j < NT_h; entries j >= NT_h and unused rows are 0.  map
+ * [B, heads, R, NT_max] fp32 (written in full).  scale <= 0 selects
+ * 1/sqrt(d).  workspace: >= veda_tile_map_workspace() bytes of device
+ * scratch, 256-byte aligned. */
+veda_status veda_tile_map_maxpool(const veda_problem* p, const void* qp, const void* kp,
+                                  const int32_t* rows, int32_t R, float scale, float* map,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------- status */
+
+/* Synchronises `stream`, then reads and clears the library's device error
+ * word (set by a kernel that gave up on a bounded wait).  Returns VEDA_OK,
+ * VEDA_ERR_TIMEOUT or VEDA_ERR_CUDA. */
+veda_status veda_sync_status(void* stream);
+
+/* Limit of every bounded wait inside the library's kernels, in nanoseconds
+ * (default 2 s; accepted range [1 us, 60 s]).  Process-wide, read at launch
+ * time.  A kernel that runs a wait out sets the device error word, drains
+ * its in-flight copies, frees its tensor memory and returns. */
+veda_status veda_set_wait_timeout_ns(uint64_t ns);
+
+/* Failure-detection self-test (no counterpart on the pages): launches one
+ * tiny kernel that waits on an mbarrier nothing ever arrives on, for at most
+ * `timeout_ns` ([1 us, 10 s]).  The following veda_sync_status(stream)
+ * must report VEDA_ERR_TIMEOUT; the context stays usable. */
+veda_status veda_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
+
+/* Thread-local text of the last failure ("" if none).  Valid until the next
+ * call on this thread. */
+const char* veda_last_error(void);
+
+/* Library version, "major.minor.patch". */
+const char* veda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VEDA_H_ */

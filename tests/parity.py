@@ -1,0 +1,92 @@
+"""Shared helpers for the parity tests: run the CUDA path through the C ABI and
+the fp64 oracle on the same seeded inputs, and compare them element by element
+with the tolerances of the tile-sparse attention contract:
+
+* permute / unpermute / idx: bit-exact (idx up to near-ties: a selection may
+  differ from the oracle's only for tiles whose exact score is within 1e-4 of
+  the k-th largest score of that row);
+* TripPool: max / min exact, mean relative 1e-5;
+* probabilities: relative 2e-5 + absolute 1e-7 (fp32 exp of fp32 scores);
+* attention output (bf16 inputs, fp32 accumulation, bf16 output): max-abs
+  1e-2 and relative L2 5e-3 against the fp64 oracle; log-sum-exp absolute 1e-3;
+* tile map: relative 1e-3 on entries >= 1e-8 (absolute 1e-11 below).
+"""
+from __future__ import annotations
+
+import math
+from typing import List, Sequence
+
+import numpy as np
+import torch
+
+from oracle import veda_oracle as O
+
+ATTN_MAX_ABS = 1e-2
+ATTN_REL_L2 = 5e-3
+LSE_ABS = 1e-3
+MEAN_REL = 1e-5
+PROBS_REL = 2e-5
+PROBS_ABS = 1e-7
+MAP_REL = 1e-3
+NEAR_TIE = 1e-4
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+def check_idx(gpu_idx: np.ndarray, ora_idx: np.ndarray, ora_scores: np.ndarray, nts: Sequence[int],
+              ks: Sequence[int], heads: Sequence[int] = None) -> int:
+    """Checks the idx contract and equality up to near-ties; returns the number of rows that differ."""
+    B, H, ntmax, kmax = gpu_idx.shape
+    heads = range(H) if heads is None else heads
+    differ = 0
+    for b in range(B):
+        for hh, h in enumerate(heads):
+            nt, k = nts[h], ks[h]
+            for i in range(ntmax):
+                g = gpu_idx[b, hh, i]
+                if i >= nt:
+                    assert np.all(g == -1), (b, h, i)
+                    continue
+                assert np.all(g[k:] == -1), (b, h, i)
+                sel = g[:k]
+                assert np.all(sel >= 0) and np.all(sel < nt), (b, h, i, sel)
+                assert np.all(np.diff(sel) > 0), (b, h, i, sel)
+                o = ora_idx[b, hh, i, :k]
+                if np.array_equal(sel, o):
+                    continue
+                differ += 1
+                s = ora_scores[b, hh, i, :nt]
+                kth = np.sort(s)[::-1][k - 1]
+                for j in set(sel.tolist()) ^ set(o.tolist()):
+                    assert abs(s[j] - kth) < NEAR_TIE, (b, h, i, j, s[j], kth)
+    return differ
+
+
+def check_attn_rows(gpu_rows: np.ndarray, ora_rows: np.ndarray, what: str = "attention"):
+    err = np.abs(gpu_rows - ora_rows)
+    max_abs = float(err.max()) if err.size else 0.0
+    rel = float(np.linalg.norm(gpu_rows - ora_rows) / max(np.linalg.norm(ora_rows), 1e-30))
+    assert max_abs <= ATTN_MAX_ABS, f"{what}: max abs error {max_abs:.3e} > {ATTN_MAX_ABS}"
+    assert rel <= ATTN_REL_L2, f"{what}: relative L2 error {rel:.3e} > {ATTN_REL_L2}"
+    return max_abs, rel
+
+
+def token_rows(grid, tiling, S, i) -> np.ndarray:
+    """Slots of tile i that hold a token (from the oracle's slot table)."""
+    tab = O.slot_table(grid, tiling)
+    return np.nonzero(tab[i * S:(i + 1) * S] >= 0)[0]
+
+
+def mlp_numpy(m) -> tuple:
+    return tuple(t.detach().cpu().to(torch.float64).numpy() for t in (m.w1, m.b1, m.w2, m.b2))
+
+
+def mlp_device(m, device="cuda") -> tuple:
+    return tuple(t.to(device).contiguous() for t in (m.w1, m.b1, m.w2, m.b2))
+
+
+def keep_f32(r: float) -> float:
+    """The keep ratio as the C ABI receives it (a C float), widened back to double."""
+    return float(np.float32(r))

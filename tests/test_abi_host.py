@@ -1,0 +1,104 @@
+"""CPU-only checks of the C-ABI library: it loads, exports every entry point
+declared in include/veda.h, and its host-side logic (layout, keep counts,
+argument validation, workspace sizes) agrees with the oracle.  No call here
+launches a kernel."""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import veda_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "veda.h")
+
+
+@pytest.fixture(scope="module")
+def V():
+    import tile_sparse_attention_head_b200 as V
+    return V
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(veda_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol(V):
+    syms = declared_symbols()
+    assert len(syms) >= 15
+    lib = ctypes.CDLL(V.LIB_PATH)
+    for s in syms:
+        assert hasattr(lib, s), s
+
+
+def test_library_is_built_for_sm100a(V):
+    # The build command pins the architecture; the library must not carry a CPU path.
+    from tile_sparse_attention_head_b200 import build
+    cmd = " ".join(build.nvcc_command())
+    assert "arch=compute_100a,code=sm_100a" in cmd
+
+
+CASES = [((4, 8, 8), 64, [(1, 8, 8), (4, 4, 4)]),
+         ((21, 30, 52), 128, [(2, 8, 8), (1, 8, 16), (8, 4, 4), (4, 4, 8)]),
+         ((21, 45, 80), 128, [(2, 8, 8), (1, 8, 16), (8, 4, 4), (4, 4, 8)]),
+         ((5, 13, 19), 64, [(1, 8, 8), (4, 4, 4), (2, 4, 8), (1, 1, 64)])]
+
+
+@pytest.mark.parametrize("grid,S,tilings", CASES)
+def test_layout_and_keep_counts_match_oracle(V, grid, S, tilings):
+    p = V.Problem(1, len(tilings), 128, S, grid, tilings)
+    nts, ntmax = O.tile_layout(grid, tilings)
+    assert p.nt_per_head == nts and p.nt_max == ntmax
+    for r in (0.01, 0.05, 0.1, 0.3, 0.5, 0.7, 1.0):
+        ks, kmax = p.keep_count(r)
+        rr = float(np.float32(r))
+        assert ks == [O.keep_count(n, rr) for n in nts]
+        assert kmax == max(ks)
+
+
+def test_invalid_arguments_are_rejected_on_the_host(V):
+    B = V.binding
+    with pytest.raises(V.VedaError) as e:
+        V.Problem(1, 1, 96, 128, (2, 2, 2), [(2, 8, 8)])
+    assert e.value.status == B.VEDA_ERR_UNSUPPORTED
+    with pytest.raises(V.VedaError) as e:
+        V.Problem(1, 1, 128, 128, (2, 2, 2), [(2, 8, 4)])        # pt*ph*pw != S
+    assert e.value.status == B.VEDA_ERR_INVALID_ARG
+    with pytest.raises(V.VedaError) as e:
+        V.Problem(1, 1, 128, 96, (2, 2, 2), [(2, 8, 6)])
+    assert e.value.status == B.VEDA_ERR_UNSUPPORTED
+    with pytest.raises(V.VedaError):
+        V.Problem(0, 1, 128, 128, (2, 2, 2), [(2, 8, 8)])
+    with pytest.raises(V.VedaError):
+        V.Problem(1, 1, 128, 128, (0, 2, 2), [(2, 8, 8)])
+    p = V.Problem(1, 1, 128, 128, (4, 8, 8), [(2, 8, 8)])
+    with pytest.raises(V.VedaError) as e:
+        p.keep_count(0.0)
+    assert e.value.status == B.VEDA_ERR_INVALID_ARG
+    with pytest.raises(V.VedaError):
+        p.keep_count(1.5)
+    lib = V.LIB
+    # NULL tensors are refused before anything touches the GPU
+    assert lib.veda_tile_permute(p.ref, None, None, None) == B.VEDA_ERR_INVALID_ARG
+    assert lib.veda_tripool(p.ref, None, None, None) == B.VEDA_ERR_INVALID_ARG
+    assert lib.veda_tile_sparse_attn(p.ref, None, None, None, None, 1, 0.0, None, None, None) == B.VEDA_ERR_INVALID_ARG
+    assert b"non-NULL" in lib.veda_last_error() or b"NULL" in lib.veda_last_error()
+    # misaligned pointers are refused too
+    assert lib.veda_tile_permute(p.ref, 8, 16, None) == B.VEDA_ERR_INVALID_ARG
+    assert lib.veda_set_wait_timeout_ns(0) == B.VEDA_ERR_INVALID_ARG
+    assert lib.veda_selftest_wait_timeout(10**12, None) == B.VEDA_ERR_INVALID_ARG
+
+
+def test_workspace_sizes(V):
+    p = V.Problem(2, 3, 64, 64, (5, 13, 19), [(1, 8, 8), (4, 4, 4), (2, 4, 8)])
+    e = 32
+    assert V.veda_score_topk_workspace(p, e) >= 4 * 2 * 2 * 3 * p.nt_max * e
+    R = 7
+    assert V.veda_tile_map_workspace(p, R) >= 4 * 2 * 3 * R * (p.nt_max * 64 + 64)
+    with pytest.raises(V.VedaError):
+        V.veda_score_topk_workspace(p, 3)

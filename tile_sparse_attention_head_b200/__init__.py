@@ -1,0 +1,12 @@
+"""B200 (sm_100a) head-aware tile-sparse attention (Veda).
+
+The C ABI lives in ``include/veda.h`` and ``libveda.so`` (built in-tree by
+``build.py``); ``binding`` is its ctypes wrapper and ``pipeline`` chains the
+calls into the per-layer inference path.  Importing this package loads the
+library and fails loudly if it is not built.
+"""
+from .binding import (  # noqa: F401
+    LIB, LIB_PATH, Problem, VedaError, make_mlp, veda_score_topk_workspace, veda_selftest_wait_timeout,
+    veda_set_wait_timeout_ns, veda_sync_status, veda_tile_map_maxpool, veda_tile_map_workspace, veda_tile_permute,
+    veda_tile_score_topk, veda_tile_sparse_attn, veda_tile_unpermute, veda_tripool, veda_version)
+from .pipeline import VedaAttention  # noqa: F401

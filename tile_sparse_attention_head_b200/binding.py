@@ -1,0 +1,256 @@
+"""ctypes binding of libveda.so (the C ABI in include/veda.h).
+
+Argument marshalling only: every function here checks tensor devices, dtypes
+and shapes, passes raw device pointers and the current CUDA stream to the
+library function of the same name, and raises ``VedaError`` on a non-zero
+status.  All computation runs in the library's CUDA kernels; there is no
+fallback of any kind -- if the library is missing, importing this module
+fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libveda.so")
+
+VEDA_OK, VEDA_ERR_INVALID_ARG, VEDA_ERR_UNSUPPORTED, VEDA_ERR_CUDA, VEDA_ERR_TIMEOUT = range(5)
+MAX_HEADS = 128
+_STATUS_NAMES = {0: "VEDA_OK", 1: "VEDA_ERR_INVALID_ARG", 2: "VEDA_ERR_UNSUPPORTED", 3: "VEDA_ERR_CUDA",
+                 4: "VEDA_ERR_TIMEOUT"}
+
+
+class VedaError(RuntimeError):
+    def __init__(self, status: int, func: str, message: str):
+        super().__init__(f"{func}: {_STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class veda_grid(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("W", ctypes.c_int32)]
+
+
+class veda_tiling(ctypes.Structure):
+    _fields_ = [("pt", ctypes.c_int32), ("ph", ctypes.c_int32), ("pw", ctypes.c_int32)]
+
+
+class veda_problem(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("heads", ctypes.c_int32), ("d", ctypes.c_int32), ("S", ctypes.c_int32),
+                ("grid", veda_grid), ("tilings", ctypes.POINTER(veda_tiling))]
+
+
+class veda_mlp(ctypes.Structure):
+    _fields_ = [("w1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("w2", ctypes.c_void_p), ("b2", ctypes.c_void_p),
+                ("hidden", ctypes.c_int32), ("e", ctypes.c_int32)]
+
+
+_P = ctypes.POINTER(veda_problem)
+_V = ctypes.c_void_p
+_I32P = ctypes.POINTER(ctypes.c_int32)
+_SIG = {
+    "veda_tile_layout": [_P, _I32P, _I32P],
+    "veda_keep_count": [_P, ctypes.c_float, _I32P, _I32P],
+    "veda_tile_permute": [_P, _V, _V, _V],
+    "veda_tile_unpermute": [_P, _V, _V, _V],
+    "veda_tripool": [_P, _V, _V, _V],
+    "veda_score_topk_workspace": [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)],
+    "veda_tile_score_topk": [_P, _V, _V, ctypes.POINTER(veda_mlp), ctypes.POINTER(veda_mlp), ctypes.c_float, _V,
+                             ctypes.c_int32, _V, _V, ctypes.c_size_t, _V],
+    "veda_tile_sparse_attn": [_P, _V, _V, _V, _V, ctypes.c_int32, ctypes.c_float, _V, _V, _V],
+    "veda_tile_map_workspace": [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)],
+    "veda_tile_map_maxpool": [_P, _V, _V, _V, ctypes.c_int32, ctypes.c_float, _V, _V, ctypes.c_size_t, _V],
+    "veda_sync_status": [_V],
+    "veda_set_wait_timeout_ns": [ctypes.c_uint64],
+    "veda_selftest_wait_timeout": [ctypes.c_uint64, _V],
+}
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libveda.so is not built ({LIB_PATH}); run tile_sparse_attention_head_b200/build.py")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, args in _SIG.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    lib.veda_last_error.restype = ctypes.c_char_p
+    lib.veda_last_error.argtypes = []
+    lib.veda_version.restype = ctypes.c_char_p
+    lib.veda_version.argtypes = []
+    return lib
+
+
+LIB = _load()
+
+
+def _check(status: int, func: str) -> None:
+    if status != VEDA_OK:
+        raise VedaError(status, func, LIB.veda_last_error().decode())
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor], name: str, dtype: Optional[torch.dtype] = None,
+         shape: Optional[Tuple[int, ...]] = None) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} (got {t.dtype})")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
+    return t.data_ptr()
+
+
+class Problem:
+    """The problem statement (B, heads, d, S, grid, per-head tilings) as the C struct."""
+
+    def __init__(self, B: int, heads: int, d: int, S: int, grid: Sequence[int],
+                 tilings: Sequence[Sequence[int]]):
+        self.B, self.heads, self.d, self.S = int(B), int(heads), int(d), int(S)
+        self.grid = tuple(int(v) for v in grid)
+        self.tilings = tuple(tuple(int(v) for v in t) for t in tilings)
+        if len(self.tilings) != self.heads:
+            raise ValueError("one tiling per head is required")
+        self._tilings_arr = (veda_tiling * max(1, self.heads))(*[veda_tiling(*t) for t in self.tilings])
+        self.c = veda_problem(self.B, self.heads, self.d, self.S, veda_grid(*self.grid),
+                              ctypes.cast(self._tilings_arr, ctypes.POINTER(veda_tiling)))
+        nts = (ctypes.c_int32 * self.heads)()
+        ntmax = ctypes.c_int32()
+        _check(LIB.veda_tile_layout(ctypes.byref(self.c), nts, ctypes.byref(ntmax)), "veda_tile_layout")
+        self.nt_per_head = list(nts)
+        self.nt_max = int(ntmax.value)
+
+    @property
+    def N(self) -> int:
+        return self.grid[0] * self.grid[1] * self.grid[2]
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
+
+    def grid_shape(self) -> Tuple[int, int, int, int]:
+        return (self.B, self.heads, self.N, self.d)
+
+    def tile_shape(self) -> Tuple[int, int, int, int]:
+        return (self.B, self.heads, self.nt_max * self.S, self.d)
+
+    def keep_count(self, keep_ratio: float):
+        ks = (ctypes.c_int32 * self.heads)()
+        kmax = ctypes.c_int32()
+        _check(LIB.veda_keep_count(self.ref, ctypes.c_float(keep_ratio), ks, ctypes.byref(kmax)), "veda_keep_count")
+        return list(ks), int(kmax.value)
+
+
+def veda_tile_permute(p: Problem, x: torch.Tensor, xp: torch.Tensor, stream=None) -> torch.Tensor:
+    _check(LIB.veda_tile_permute(p.ref, _ptr(x, "x", torch.bfloat16, p.grid_shape()),
+                                 _ptr(xp, "xp", torch.bfloat16, p.tile_shape()), _stream(stream)),
+           "veda_tile_permute")
+    return xp
+
+
+def veda_tile_unpermute(p: Problem, xp: torch.Tensor, x: torch.Tensor, stream=None) -> torch.Tensor:
+    _check(LIB.veda_tile_unpermute(p.ref, _ptr(xp, "xp", torch.bfloat16, p.tile_shape()),
+                                   _ptr(x, "x", torch.bfloat16, p.grid_shape()), _stream(stream)),
+           "veda_tile_unpermute")
+    return x
+
+
+def veda_tripool(p: Problem, xp: torch.Tensor, desc: torch.Tensor, stream=None) -> torch.Tensor:
+    _check(LIB.veda_tripool(p.ref, _ptr(xp, "xp", torch.bfloat16, p.tile_shape()),
+                            _ptr(desc, "desc", torch.float32, (p.B, p.heads, p.nt_max, 3 * p.d)), _stream(stream)),
+           "veda_tripool")
+    return desc
+
+
+def veda_score_topk_workspace(p: Problem, e: int) -> int:
+    n = ctypes.c_size_t()
+    _check(LIB.veda_score_topk_workspace(p.ref, int(e), ctypes.byref(n)), "veda_score_topk_workspace")
+    return int(n.value)
+
+
+def make_mlp(w1: torch.Tensor, b1: torch.Tensor, w2: torch.Tensor, b2: torch.Tensor) -> veda_mlp:
+    """C struct for one set of per-head estimator weights (fp32 device tensors)."""
+    heads, hidden, _ = w1.shape
+    e = w2.shape[1]
+    for t, n in ((w1, "w1"), (b1, "b1"), (w2, "w2"), (b2, "b2")):
+        _ptr(t, n, torch.float32)
+    if tuple(b1.shape) != (heads, hidden) or tuple(w2.shape) != (heads, e, hidden) or tuple(b2.shape) != (heads, e):
+        raise ValueError("estimator weight shapes must be w1 [h,hid,3d], b1 [h,hid], w2 [h,e,hid], b2 [h,e]")
+    return veda_mlp(w1.data_ptr(), b1.data_ptr(), w2.data_ptr(), b2.data_ptr(), int(hidden), int(e))
+
+
+def veda_tile_score_topk(p: Problem, desc_q: torch.Tensor, desc_k: torch.Tensor, mlp_q: veda_mlp, mlp_k: veda_mlp,
+                         keep_ratio: float, idx: torch.Tensor, probs: Optional[torch.Tensor],
+                         workspace: torch.Tensor, stream=None) -> torch.Tensor:
+    dshape = (p.B, p.heads, p.nt_max, 3 * p.d)
+    k_max = int(idx.shape[-1])
+    _check(LIB.veda_tile_score_topk(
+        p.ref, _ptr(desc_q, "desc_q", torch.float32, dshape), _ptr(desc_k, "desc_k", torch.float32, dshape),
+        ctypes.byref(mlp_q), ctypes.byref(mlp_k), ctypes.c_float(keep_ratio),
+        _ptr(idx, "idx", torch.int32, (p.B, p.heads, p.nt_max, k_max)), k_max,
+        _ptr(probs, "probs", torch.float32, (p.B, p.heads, p.nt_max, p.nt_max)),
+        _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)),
+        "veda_tile_score_topk")
+    return idx
+
+
+def veda_tile_sparse_attn(p: Problem, qp: torch.Tensor, kp: torch.Tensor, vp: torch.Tensor, idx: torch.Tensor,
+                          op: torch.Tensor, lse: Optional[torch.Tensor] = None, scale: float = 0.0,
+                          stream=None) -> torch.Tensor:
+    ts = p.tile_shape()
+    k_max = int(idx.shape[-1])
+    _check(LIB.veda_tile_sparse_attn(
+        p.ref, _ptr(qp, "qp", torch.bfloat16, ts), _ptr(kp, "kp", torch.bfloat16, ts),
+        _ptr(vp, "vp", torch.bfloat16, ts), _ptr(idx, "idx", torch.int32, (p.B, p.heads, p.nt_max, k_max)), k_max,
+        ctypes.c_float(scale), _ptr(op, "op", torch.bfloat16, ts),
+        _ptr(lse, "lse", torch.float32, (p.B, p.heads, p.nt_max * p.S)), _stream(stream)),
+        "veda_tile_sparse_attn")
+    return op
+
+
+def veda_tile_map_workspace(p: Problem, R: int) -> int:
+    n = ctypes.c_size_t()
+    _check(LIB.veda_tile_map_workspace(p.ref, int(R), ctypes.byref(n)), "veda_tile_map_workspace")
+    return int(n.value)
+
+
+def veda_tile_map_maxpool(p: Problem, qp: torch.Tensor, kp: torch.Tensor, rows: torch.Tensor, out: torch.Tensor,
+                          workspace: torch.Tensor, scale: float = 0.0, stream=None) -> torch.Tensor:
+    ts = p.tile_shape()
+    R = int(rows.shape[-1])
+    _check(LIB.veda_tile_map_maxpool(
+        p.ref, _ptr(qp, "qp", torch.bfloat16, ts), _ptr(kp, "kp", torch.bfloat16, ts),
+        _ptr(rows, "rows", torch.int32, (p.B * p.heads, R)), R, ctypes.c_float(scale),
+        _ptr(out, "map", torch.float32, (p.B, p.heads, R, p.nt_max)), _ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "veda_tile_map_maxpool")
+    return out
+
+
+def veda_sync_status(stream=None) -> None:
+    _check(LIB.veda_sync_status(_stream(stream)), "veda_sync_status")
+
+
+def veda_set_wait_timeout_ns(ns: int) -> None:
+    _check(LIB.veda_set_wait_timeout_ns(int(ns)), "veda_set_wait_timeout_ns")
+
+
+def veda_selftest_wait_timeout(timeout_ns: int, stream=None) -> None:
+    _check(LIB.veda_selftest_wait_timeout(int(timeout_ns), _stream(stream)), "veda_selftest_wait_timeout")
+
+
+def veda_version() -> str:
+    return LIB.veda_version().decode()

@@ -1,0 +1,64 @@
+// Launchers of the sm_100a kernels (internal to the library; the public
+// surface is include/veda.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "veda_common.cuh"
+
+namespace veda {
+
+struct EstimatorWeights {
+  const float* w1;
+  const float* b1;
+  const float* w2;
+  const float* b2;
+};
+
+struct TopkArgs {
+  int32_t* idx;
+  float* probs;
+  int32_t k_max;
+  int32_t k_per_head[VEDA_MAX_HEADS];
+};
+
+struct AttnArgs {
+  const int32_t* idx;
+  int32_t k_max;
+  float scale_log2;   // softmax scale * log2(e)
+  void* op;           // bf16 [B, heads, NT_max*S, d]
+  float* lse;         // fp32 [B, heads, NT_max*S] or null
+  uint64_t timeout_ns;
+};
+
+struct MapArgs {
+  const int32_t* rows;  // [B*heads, R]
+  int32_t R;
+  float scale_log2;
+  float* rowmax;        // scratch [B*heads, R, NT_max, S]  (scaled, log2 domain)
+  float* lse2;          // scratch [B*heads, R, S]          (log2 domain)
+  float* map;           // [B, heads, R, NT_max]
+  uint64_t timeout_ns;
+};
+
+cudaError_t launch_permute(const Geometry& G, const void* x, void* xp, cudaStream_t s, int sms);
+cudaError_t launch_unpermute(const Geometry& G, const void* xp, void* x, cudaStream_t s, int sms);
+cudaError_t launch_tripool(const Geometry& G, const void* xp, float* desc, cudaStream_t s);
+
+size_t estimator_smem_bytes(int d, int hidden);
+void score_topk_config(int ntmax, int e, int* qb, int* ntpad, size_t* smem);
+cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const float* desc_k,
+                              const EstimatorWeights& wq, const EstimatorWeights& wk, int hidden,
+                              int e, float* phi, const TopkArgs& args, cudaStream_t s);
+
+cudaError_t launch_sparse_attn(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,
+                               const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
+
+cudaError_t launch_tile_map(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,
+                            const MapArgs& a, cudaStream_t s);
+
+cudaError_t launch_timeout_selftest(uint64_t timeout_ns, cudaStream_t s);
+
+}  // namespace veda

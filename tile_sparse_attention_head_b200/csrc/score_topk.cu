@@ -1,0 +1,311 @@
+// Distilled tile scoring and top-k selection (section 2.1 of the Veda summary:
+// a head-specific MLP maps each tile's TripPool descriptor to a feature;
+// tile scores form a row-wise distribution over K tiles; section 4 / news
+// page: keep the top ~5-10% of tiles).
+//
+// Two kernels:
+//   estimator_kernel  phi = W2 relu(W1 desc + b1) + b2 for every Q and K tile,
+//                     fp32 on the CUDA cores, written to the workspace;
+//   score_topk_kernel per block of Q-tile rows: s = phi_q phi_k^T / sqrt(e)
+//                     into shared memory, optional row softmax, then an exact
+//                     radix select of the k-th largest score per row and an
+//                     ascending compaction of the winners.
+// Scores stay fp32 end to end so that selections only differ from an exact
+// evaluation on genuine near-ties.
+#include "veda_common.cuh"
+#include "kernels.h"
+
+namespace veda {
+
+constexpr int kEstTiles = 32;     // tiles per estimator CTA
+constexpr int kEstThreads = 256;
+constexpr int kEstChunk = 32;     // input channels staged per step
+
+// grid: (ceil(NT_max / 32), B*heads, 2)  z = 0: Q descriptors, z = 1: K.
+__global__ void __launch_bounds__(kEstThreads)
+    estimator_kernel(const __grid_constant__ Geometry G, const float* __restrict__ desc_q,
+                     const float* __restrict__ desc_k, EstimatorWeights wq, EstimatorWeights wk,
+                     int hidden, int e, float* __restrict__ phi) {
+  extern __shared__ float sm[];
+  const int in_dim = 3 * G.d;
+  const int which = blockIdx.z;
+  const int bh = blockIdx.y;
+  const int h = bh % G.heads;
+  const int nt = G.g[h].nt;
+  const int j0 = blockIdx.x * kEstTiles;
+  if (j0 >= nt) return;
+  const int ntile = min(kEstTiles, nt - j0);
+  const EstimatorWeights& w = which ? wk : wq;
+  const float* desc = (which ? desc_k : desc_q) + ((long long)bh * G.ntmax + j0) * in_dim;
+  const float* W1 = w.w1 + (long long)h * hidden * in_dim;
+  const float* B1 = w.b1 + (long long)h * hidden;
+  const float* W2 = w.w2 + (long long)h * e * hidden;
+  const float* B2 = w.b2 + (long long)h * e;
+
+  float* s_desc = sm;                                  // [32][in_dim]
+  float* s_w1 = s_desc + kEstTiles * in_dim;           // [hidden][33]
+  float* s_hid = s_w1 + hidden * (kEstChunk + 1);      // [32][hidden]
+  const int tid = threadIdx.x;
+
+  for (int i = tid; i < kEstTiles * in_dim; i += kEstThreads) {
+    const int t = i / in_dim;
+    s_desc[i] = (t < ntile) ? desc[i] : 0.f;
+  }
+
+  // Layer 1: each thread owns hidden units u = tid, tid + 256 (hidden <= 512).
+  float acc[2][kEstTiles];
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int t = 0; t < kEstTiles; ++t) acc[a][t] = 0.f;
+
+  for (int c0 = 0; c0 < in_dim; c0 += kEstChunk) {
+    __syncthreads();
+    for (int i = tid; i < hidden * kEstChunk; i += kEstThreads) {
+      const int u = i / kEstChunk, c = i % kEstChunk;
+      s_w1[u * (kEstChunk + 1) + c] = W1[(long long)u * in_dim + c0 + c];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+      const int u = tid + a * kEstThreads;
+      if (u < hidden) {
+        for (int c = 0; c < kEstChunk; ++c) {
+          const float wv = s_w1[u * (kEstChunk + 1) + c];
+#pragma unroll
+          for (int t = 0; t < kEstTiles; ++t) acc[a][t] = fmaf(s_desc[t * in_dim + c0 + c], wv, acc[a][t]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < 2; ++a) {
+    const int u = tid + a * kEstThreads;
+    if (u < hidden) {
+      const float bb = B1[u];
+#pragma unroll
+      for (int t = 0; t < kEstTiles; ++t) s_hid[t * hidden + u] = fmaxf(acc[a][t] + bb, 0.f);
+    }
+  }
+  __syncthreads();
+
+  // Layer 2: kEstTiles * e outputs spread over the block.
+  float* out = phi + (((long long)which * G.B * G.heads + bh) * G.ntmax + j0) * e;
+  for (int i = tid; i < ntile * e; i += kEstThreads) {
+    const int t = i / e, o = i % e;
+    const float* w2row = W2 + (long long)o * hidden;
+    const float* hrow = s_hid + t * hidden;
+    float acc2 = 0.f;
+    for (int k = 0; k < hidden; ++k) acc2 = fmaf(hrow[k], __ldg(w2row + k), acc2);
+    out[(long long)t * e + o] = acc2 + B2[o];
+  }
+}
+
+size_t estimator_smem_bytes(int d, int hidden) {
+  return sizeof(float) * ((size_t)kEstTiles * 3 * d + (size_t)hidden * (kEstChunk + 1) +
+                          (size_t)kEstTiles * hidden);
+}
+
+// Order-preserving map fp32 -> uint32 (larger float <-> larger key).
+__device__ __forceinline__ uint32_t float_key(float f) {
+  const uint32_t u = __float_as_uint(f + 0.0f);  // -0 -> +0: equal scores get equal keys
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+constexpr int kScoreThreads = 256;
+constexpr int kKChunk = 64;        // K tiles staged per step
+
+// grid: (ceil(NT_max / qb), B*heads).  Shared memory: scores [qb][ntmax_pad],
+// phi_q [qb][e], phi_k chunk [64][e+1], radix histograms [8][256].
+__global__ void __launch_bounds__(kScoreThreads)
+    score_topk_kernel(const __grid_constant__ Geometry G, const float* __restrict__ phi, int e,
+                      int qb, int ntpad, const __grid_constant__ TopkArgs args) {
+  extern __shared__ float sm[];
+  const int bh = blockIdx.y;
+  const int h = bh % G.heads;
+  const int nt = G.g[h].nt;
+  const int i0 = blockIdx.x * qb;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int k = args.k_per_head[h];
+  int32_t* idx_base = args.idx + ((long long)bh * G.ntmax) * args.k_max;
+  float* probs_base = args.probs ? args.probs + ((long long)bh * G.ntmax) * G.ntmax : nullptr;
+
+  if (i0 >= nt) {
+    // Rows of tiles that do not exist in this head: idx -1, probs 0.
+    for (int r = 0; r < qb; ++r) {
+      const int i = i0 + r;
+      if (i >= G.ntmax) break;
+      for (int c = tid; c < args.k_max; c += kScoreThreads) idx_base[(long long)i * args.k_max + c] = -1;
+      if (probs_base)
+        for (int c = tid; c < G.ntmax; c += kScoreThreads) probs_base[(long long)i * G.ntmax + c] = 0.f;
+    }
+    return;
+  }
+  const int nrows = min(qb, nt - i0);
+  float* s_scores = sm;                            // [qb][ntpad]
+  float* s_phiq = s_scores + qb * ntpad;           // [qb][e]
+  float* s_phik = s_phiq + qb * e;                 // [64][e+1]
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(s_phik + kKChunk * (e + 1));  // [8][256]
+
+  const float* phq = phi + ((long long)bh * G.ntmax + i0) * e;
+  const float* phk = phi + (((long long)G.B * G.heads + bh) * G.ntmax) * e;
+  for (int i = tid; i < qb * e; i += kScoreThreads) s_phiq[i] = (i / e < nrows) ? phq[i] : 0.f;
+  const float inv_sqrt_e = rsqrtf((float)e);
+
+  // Scores: thread -> column c = tid % 64 of the chunk, rows rg, rg+4, ...
+  const int c_local = tid % kKChunk, rg = tid / kKChunk;
+  for (int jc = 0; jc < nt; jc += kKChunk) {
+    __syncthreads();
+    const int ncols = min(kKChunk, nt - jc);
+    for (int i = tid; i < kKChunk * e; i += kScoreThreads) {
+      const int jj = i / e, cc = i % e;
+      s_phik[jj * (e + 1) + cc] = (jj < ncols) ? phk[(long long)(jc + jj) * e + cc] : 0.f;
+    }
+    __syncthreads();
+    if (c_local < ncols) {
+      for (int r = rg; r < nrows; r += kScoreThreads / kKChunk) {
+        const float* a = s_phiq + r * e;
+        const float* b = s_phik + c_local * (e + 1);
+        float acc = 0.f;
+        for (int cc = 0; cc < e; ++cc) acc = fmaf(a[cc], b[cc], acc);
+        s_scores[r * ntpad + jc + c_local] = acc * inv_sqrt_e;
+      }
+    }
+  }
+  __syncthreads();
+
+  uint32_t* hist = s_hist + warp * 256;
+  for (int r = warp; r < qb; r += kScoreThreads / 32) {
+    const int i = i0 + r;
+    if (i >= G.ntmax) break;
+    int32_t* irow = idx_base + (long long)i * args.k_max;
+    if (r >= nrows) {
+      for (int c = lane; c < args.k_max; c += 32) irow[c] = -1;
+      if (probs_base)
+        for (int c = lane; c < G.ntmax; c += 32) probs_base[(long long)i * G.ntmax + c] = 0.f;
+      continue;
+    }
+    const float* srow = s_scores + r * ntpad;
+
+    // Optional row softmax.
+    if (probs_base) {
+      float m = -INFINITY;
+      for (int c = lane; c < nt; c += 32) m = fmaxf(m, srow[c]);
+#pragma unroll
+      for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      float sum = 0.f;
+      for (int c = lane; c < nt; c += 32) sum += expf(srow[c] - m);
+#pragma unroll
+      for (int off = 16; off; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      const float inv = 1.0f / sum;
+      float* prow = probs_base + (long long)i * G.ntmax;
+      for (int c = lane; c < G.ntmax; c += 32) prow[c] = (c < nt) ? expf(srow[c] - m) * inv : 0.f;
+    }
+
+    // Radix select: find the k-th largest key, 8 bits per pass from the top.
+    uint32_t prefix = 0, pmask = 0;
+    int remaining = k;
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int b = lane; b < 256; b += 32) hist[b] = 0;
+      __syncwarp();
+      for (int c = lane; c < nt; c += 32) {
+        const uint32_t key = float_key(srow[c]);
+        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
+      __syncwarp();
+      // Lane L owns bins 255-8L .. 248-8L (descending); scan counts from the top.
+      uint32_t cnt[8];
+      uint32_t local = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        cnt[q] = hist[255 - (lane * 8 + q)];
+        local += cnt[q];
+      }
+      uint32_t incl = local;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      const uint32_t excl = incl - local;
+      // The bin holding the remaining-th largest key: excl + partial < remaining <= excl + partial + cnt.
+      int found_bin = -1;
+      uint32_t above = 0;
+      if ((uint32_t)remaining > excl && (uint32_t)remaining <= incl) {
+        uint32_t run = excl;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (found_bin < 0 && (uint32_t)remaining <= run + cnt[q]) {
+            found_bin = 255 - (lane * 8 + q);
+            above = run;
+          }
+          run += cnt[q];
+        }
+      }
+      const unsigned who = __ballot_sync(0xffffffffu, found_bin >= 0);
+      const int src = __ffs(who) - 1;
+      found_bin = __shfl_sync(0xffffffffu, found_bin, src);
+      above = __shfl_sync(0xffffffffu, above, src);
+      remaining -= (int)above;
+      prefix |= (uint32_t)found_bin << shift;
+      pmask |= 255u << shift;
+      __syncwarp();
+    }
+    // prefix = k-th largest key; take every key above it and the first
+    // `remaining` keys equal to it (smallest tile indices), in ascending order.
+    int out = 0, eq_taken = 0;
+    for (int c0 = 0; c0 < nt; c0 += 32) {
+      const int c = c0 + lane;
+      uint32_t key = 0;
+      const bool in = c < nt;
+      if (in) key = float_key(srow[c]);
+      const bool gt = in && key > prefix;
+      const bool eq = in && key == prefix;
+      const unsigned eqmask = __ballot_sync(0xffffffffu, eq);
+      const int eq_before = __popc(eqmask & ((1u << lane) - 1u));
+      const bool take = gt || (eq && eq_taken + eq_before < remaining);
+      const unsigned tmask = __ballot_sync(0xffffffffu, take);
+      const int pos = out + __popc(tmask & ((1u << lane) - 1u));
+      if (take && pos < k) irow[pos] = c;
+      out += __popc(tmask);
+      eq_taken += __popc(eqmask);
+    }
+    for (int c = k + lane; c < args.k_max; c += 32) irow[c] = -1;
+  }
+}
+
+cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const float* desc_k,
+                              const EstimatorWeights& wq, const EstimatorWeights& wk, int hidden,
+                              int e, float* phi, const TopkArgs& args, cudaStream_t s) {
+  const size_t est_smem = estimator_smem_bytes(G.d, hidden);
+  cudaError_t err = cudaFuncSetAttribute(estimator_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)est_smem);
+  if (err != cudaSuccess) return err;
+  dim3 g1((G.ntmax + kEstTiles - 1) / kEstTiles, G.B * G.heads, 2);
+  estimator_kernel<<<g1, kEstThreads, est_smem, s>>>(G, desc_q, desc_k, wq, wk, hidden, e, phi);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+
+  int qb, ntpad;
+  size_t smem;
+  score_topk_config(G.ntmax, e, &qb, &ntpad, &smem);
+  err = cudaFuncSetAttribute(score_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  dim3 g2((G.ntmax + qb - 1) / qb, G.B * G.heads);
+  score_topk_kernel<<<g2, kScoreThreads, smem, s>>>(G, phi, e, qb, ntpad, args);
+  return cudaGetLastError();
+}
+
+// Rows per CTA so that the score block fits in ~160 KB of shared memory.
+void score_topk_config(int ntmax, int e, int* qb, int* ntpad, size_t* smem) {
+  const int pad = (ntmax + 3) & ~3;
+  int rows = (int)((160 * 1024) / (4 * (size_t)pad));
+  if (rows > 16) rows = 16;
+  if (rows < 1) rows = 1;
+  *qb = rows;
+  *ntpad = pad;
+  *smem = sizeof(float) * ((size_t)rows * pad + (size_t)rows * e + (size_t)kKChunk * (e + 1)) +
+          sizeof(uint32_t) * 8 * 256;
+}
+
+}  // namespace veda

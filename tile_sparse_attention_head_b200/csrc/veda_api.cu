@@ -1,0 +1,386 @@
+// C ABI of the library (declared in include/veda.h): host-side validation,
+// geometry set-up, TMA descriptor encoding and kernel launches.  Built as one
+// translation unit together with the kernel sources so the device error word
+// needs no separate device link.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "veda_common.cuh"
+#include "kernels.h"
+
+#include "permute_tripool.cu"
+#include "score_topk.cu"
+#include "sparse_attn.cu"
+#include "tile_map.cu"
+
+namespace veda {
+namespace {
+
+thread_local char g_last_error[512] = "";
+uint64_t g_timeout_ns = 2000000000ull;  // bounded-wait limit for every kernel (2 s)
+
+veda_status fail(veda_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+veda_status ok() {
+  g_last_error[0] = '\0';
+  return VEDA_OK;
+}
+
+veda_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(VEDA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Validates the problem statement and fills the kernels' geometry block.
+veda_status make_geometry(const veda_problem* p, Geometry* G) {
+  if (p == nullptr) return fail(VEDA_ERR_INVALID_ARG, "problem is NULL");
+  if (p->B < 1) return fail(VEDA_ERR_INVALID_ARG, "B must be >= 1 (got %d)", p->B);
+  if (p->heads < 1 || p->heads > VEDA_MAX_HEADS)
+    return fail(VEDA_ERR_INVALID_ARG, "heads must be in [1, %d] (got %d)", VEDA_MAX_HEADS, p->heads);
+  if (p->grid.T < 1 || p->grid.H < 1 || p->grid.W < 1)
+    return fail(VEDA_ERR_INVALID_ARG, "grid dimensions must be >= 1 (got %d x %d x %d)", p->grid.T,
+                p->grid.H, p->grid.W);
+  if (p->d != 64 && p->d != 128) return fail(VEDA_ERR_UNSUPPORTED, "head dim d must be 64 or 128 (got %d)", p->d);
+  if (p->S != 64 && p->S != 128) return fail(VEDA_ERR_UNSUPPORTED, "tile size S must be 64 or 128 (got %d)", p->S);
+  if (p->tilings == nullptr) return fail(VEDA_ERR_INVALID_ARG, "tilings is NULL");
+  const long long N = (long long)p->grid.T * p->grid.H * p->grid.W;
+  if (N > (1LL << 30)) return fail(VEDA_ERR_INVALID_ARG, "grid has too many tokens (%lld)", N);
+  std::memset(G, 0, sizeof(*G));
+  G->B = p->B;
+  G->heads = p->heads;
+  G->d = p->d;
+  G->S = p->S;
+  G->T = p->grid.T;
+  G->H = p->grid.H;
+  G->W = p->grid.W;
+  G->N = (int)N;
+  int ntmax = 0;
+  for (int h = 0; h < p->heads; ++h) {
+    const veda_tiling t = p->tilings[h];
+    if (t.pt < 1 || t.ph < 1 || t.pw < 1 || t.pt > 4096 || t.ph > 4096 || t.pw > 4096)
+      return fail(VEDA_ERR_INVALID_ARG, "head %d: tiling factors must be >= 1", h);
+    if ((long long)t.pt * t.ph * t.pw != p->S)
+      return fail(VEDA_ERR_INVALID_ARG, "head %d: pt*ph*pw = %d*%d*%d must equal S = %d", h, t.pt, t.ph,
+                  t.pw, p->S);
+    HeadGeom& g = G->g[h];
+    g.pt = (int16_t)t.pt;
+    g.ph = (int16_t)t.ph;
+    g.pw = (int16_t)t.pw;
+    const int a = ceil_div(p->grid.T, t.pt), b = ceil_div(p->grid.H, t.ph), c = ceil_div(p->grid.W, t.pw);
+    if (a > 32767 || b > 32767 || c > 32767) return fail(VEDA_ERR_INVALID_ARG, "head %d: too many tiles", h);
+    g.nTt = (int16_t)a;
+    g.nTh = (int16_t)b;
+    g.nTw = (int16_t)c;
+    g.nt = a * b * c;
+    if (g.nt > ntmax) ntmax = g.nt;
+  }
+  G->ntmax = ntmax;
+  const long long rows = (long long)p->B * p->heads * ntmax * p->S;
+  if (rows >= (1LL << 31)) return fail(VEDA_ERR_INVALID_ARG, "B*heads*NT_max*S = %lld rows exceeds 2^31", rows);
+  if ((long long)p->B * p->heads * N >= (1LL << 31))
+    return fail(VEDA_ERR_INVALID_ARG, "B*heads*N exceeds 2^31 rows");
+  return VEDA_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D view [rows, d] of a tile-major bf16 tensor, boxes of 64 channels x S rows,
+// 128-byte swizzle (the layout the tcgen05 descriptors expect).
+veda_status encode_tile_major(const Geometry& G, const void* ptr, CUtensorMap* out) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {(cuuint64_t)G.d, (cuuint64_t)G.B * G.heads * G.ntmax * G.S};
+  const cuuint64_t strides[1] = {(cuuint64_t)G.d * 2};
+  const cuuint32_t box[2] = {64u, (cuuint32_t)G.S};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return VEDA_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t score_ws_bytes(const Geometry& G, int e) {
+  return round256(sizeof(float) * 2 * (size_t)G.B * G.heads * G.ntmax * e);
+}
+
+size_t map_rowmax_bytes(const Geometry& G, int R) {
+  return round256(sizeof(float) * (size_t)G.B * G.heads * R * G.ntmax * G.S);
+}
+
+size_t map_ws_bytes(const Geometry& G, int R) {
+  return map_rowmax_bytes(G, R) + round256(sizeof(float) * (size_t)G.B * G.heads * R * G.S);
+}
+
+veda_status keep_counts(const Geometry& G, float r, int32_t* k, int32_t* kmax) {
+  if (!(r > 0.f && r <= 1.f)) return fail(VEDA_ERR_INVALID_ARG, "keep_ratio must be in (0, 1] (got %g)", (double)r);
+  int m = 0;
+  for (int h = 0; h < G.heads; ++h) {
+    const int nt = G.g[h].nt;
+    long long kk = (long long)std::floor((double)r * nt + 0.5);
+    if (kk > nt) kk = nt;
+    if (kk < 1) kk = 1;
+    if (k) k[h] = (int32_t)kk;
+    if (kk > m) m = (int)kk;
+  }
+  if (kmax) *kmax = m;
+  return VEDA_OK;
+}
+
+}  // namespace
+}  // namespace veda
+
+using namespace veda;
+
+extern "C" {
+
+const char* veda_last_error(void) { return g_last_error; }
+
+const char* veda_version(void) { return "0.1.0"; }
+
+veda_status veda_tile_layout(const veda_problem* p, int32_t* nt_per_head, int32_t* nt_max) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (nt_per_head)
+    for (int h = 0; h < G.heads; ++h) nt_per_head[h] = G.g[h].nt;
+  if (nt_max) *nt_max = G.ntmax;
+  return ok();
+}
+
+veda_status veda_keep_count(const veda_problem* p, float keep_ratio, int32_t* k_per_head, int32_t* k_max) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if ((s = keep_counts(G, keep_ratio, k_per_head, k_max)) != VEDA_OK) return s;
+  return ok();
+}
+
+veda_status veda_tile_permute(const veda_problem* p, const void* x, void* xp, void* stream) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (!x || !xp) return fail(VEDA_ERR_INVALID_ARG, "x and xp must be non-NULL");
+  if (!aligned16(x) || !aligned16(xp)) return fail(VEDA_ERR_INVALID_ARG, "x and xp must be 16-byte aligned");
+  cudaError_t e = launch_permute(G, x, xp, (cudaStream_t)stream, sm_count());
+  if (e != cudaSuccess) return cuda_fail(e, "veda_tile_permute");
+  return ok();
+}
+
+veda_status veda_tile_unpermute(const veda_problem* p, const void* xp, void* x, void* stream) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (!x || !xp) return fail(VEDA_ERR_INVALID_ARG, "x and xp must be non-NULL");
+  if (!aligned16(x) || !aligned16(xp)) return fail(VEDA_ERR_INVALID_ARG, "x and xp must be 16-byte aligned");
+  cudaError_t e = launch_unpermute(G, xp, x, (cudaStream_t)stream, sm_count());
+  if (e != cudaSuccess) return cuda_fail(e, "veda_tile_unpermute");
+  return ok();
+}
+
+veda_status veda_tripool(const veda_problem* p, const void* xp, float* desc, void* stream) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (!xp || !desc) return fail(VEDA_ERR_INVALID_ARG, "xp and desc must be non-NULL");
+  if (!aligned16(xp) || !aligned16(desc)) return fail(VEDA_ERR_INVALID_ARG, "xp and desc must be 16-byte aligned");
+  cudaError_t e = launch_tripool(G, xp, desc, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "veda_tripool");
+  return ok();
+}
+
+veda_status veda_score_topk_workspace(const veda_problem* p, int32_t e, size_t* bytes) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (e < 4 || e > 128 || e % 4) return fail(VEDA_ERR_INVALID_ARG, "e must be a multiple of 4 in [4, 128] (got %d)", e);
+  if (!bytes) return fail(VEDA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = score_ws_bytes(G, e);
+  return ok();
+}
+
+static veda_status check_mlp(const veda_mlp* m, const char* which) {
+  if (!m) return fail(VEDA_ERR_INVALID_ARG, "%s estimator is NULL", which);
+  if (!m->w1 || !m->b1 || !m->w2 || !m->b2) return fail(VEDA_ERR_INVALID_ARG, "%s estimator has a NULL weight", which);
+  if (m->hidden < 1 || m->hidden > 512) return fail(VEDA_ERR_INVALID_ARG, "hidden must be in [1, 512] (got %d)", m->hidden);
+  if (m->e < 4 || m->e > 128 || m->e % 4) return fail(VEDA_ERR_INVALID_ARG, "e must be a multiple of 4 in [4, 128] (got %d)", m->e);
+  return VEDA_OK;
+}
+
+veda_status veda_tile_score_topk(const veda_problem* p, const float* desc_q, const float* desc_k,
+                                 const veda_mlp* mlp_q, const veda_mlp* mlp_k, float keep_ratio, int32_t* idx,
+                                 int32_t k_max, float* probs, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if ((s = check_mlp(mlp_q, "q")) != VEDA_OK || (s = check_mlp(mlp_k, "k")) != VEDA_OK) return s;
+  if (mlp_q->hidden != mlp_k->hidden || mlp_q->e != mlp_k->e)
+    return fail(VEDA_ERR_INVALID_ARG, "q and k estimators must have the same hidden and e");
+  if (!desc_q || !desc_k || !idx || !workspace) return fail(VEDA_ERR_INVALID_ARG, "NULL tensor argument");
+  if (!aligned16(desc_q) || !aligned16(desc_k) || !aligned16(idx) || (probs && !aligned16(probs)))
+    return fail(VEDA_ERR_INVALID_ARG, "tensor arguments must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(VEDA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const int e = mlp_q->e, hidden = mlp_q->hidden;
+  if (workspace_bytes < score_ws_bytes(G, e))
+    return fail(VEDA_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, score_ws_bytes(G, e));
+  TopkArgs args;
+  std::memset(&args, 0, sizeof(args));
+  int32_t kmax_needed = 0;
+  if ((s = keep_counts(G, keep_ratio, args.k_per_head, &kmax_needed)) != VEDA_OK) return s;
+  if (k_max < kmax_needed) return fail(VEDA_ERR_INVALID_ARG, "k_max = %d is below the largest keep count %d", k_max, kmax_needed);
+  int qb, ntpad;
+  size_t smem;
+  score_topk_config(G.ntmax, e, &qb, &ntpad, &smem);
+  if (smem > 227 * 1024 || estimator_smem_bytes(G.d, hidden) > 227 * 1024)
+    return fail(VEDA_ERR_UNSUPPORTED, "NT_max = %d / hidden = %d exceed the shared-memory budget", G.ntmax, hidden);
+  args.idx = idx;
+  args.probs = probs;
+  args.k_max = k_max;
+  EstimatorWeights wq{mlp_q->w1, mlp_q->b1, mlp_q->w2, mlp_q->b2};
+  EstimatorWeights wk{mlp_k->w1, mlp_k->b1, mlp_k->w2, mlp_k->b2};
+  cudaError_t ce = launch_score_topk(G, desc_q, desc_k, wq, wk, hidden, e, static_cast<float*>(workspace), args,
+                                     (cudaStream_t)stream);
+  if (ce != cudaSuccess) return cuda_fail(ce, "veda_tile_score_topk");
+  return ok();
+}
+
+veda_status veda_tile_sparse_attn(const veda_problem* p, const void* qp, const void* kp, const void* vp,
+                                  const int32_t* idx, int32_t k_max, float scale, void* op, float* lse,
+                                  void* stream) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (!qp || !kp || !vp || !idx || !op) return fail(VEDA_ERR_INVALID_ARG, "NULL tensor argument");
+  if (!aligned16(qp) || !aligned16(kp) || !aligned16(vp) || !aligned16(op) || !aligned16(idx) ||
+      (lse && !aligned16(lse)))
+    return fail(VEDA_ERR_INVALID_ARG, "tensor arguments must be 16-byte aligned");
+  if (k_max < 1) return fail(VEDA_ERR_INVALID_ARG, "k_max must be >= 1 (got %d)", k_max);
+  if (!(std::isfinite(scale))) return fail(VEDA_ERR_INVALID_ARG, "scale must be finite");
+  if (sparse_attn_smem_bytes(G.d, G.S, k_max) > 227 * 1024)
+    return fail(VEDA_ERR_UNSUPPORTED, "k_max = %d exceeds the shared-memory budget", k_max);
+  CUtensorMap tq, tk, tv;
+  if ((s = encode_tile_major(G, qp, &tq)) != VEDA_OK || (s = encode_tile_major(G, kp, &tk)) != VEDA_OK ||
+      (s = encode_tile_major(G, vp, &tv)) != VEDA_OK)
+    return s;
+  AttnArgs a;
+  a.idx = idx;
+  a.k_max = k_max;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)G.d);
+  a.scale_log2 = sc * 1.4426950408889634f;
+  a.op = op;
+  a.lse = lse;
+  a.timeout_ns = g_timeout_ns;
+  cudaError_t e = launch_sparse_attn(G, tq, tk, tv, a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "veda_tile_sparse_attn");
+  return ok();
+}
+
+veda_status veda_tile_map_workspace(const veda_problem* p, int32_t R, size_t* bytes) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (R < 1) return fail(VEDA_ERR_INVALID_ARG, "R must be >= 1 (got %d)", R);
+  if (!bytes) return fail(VEDA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = map_ws_bytes(G, R);
+  return ok();
+}
+
+veda_status veda_tile_map_maxpool(const veda_problem* p, const void* qp, const void* kp, const int32_t* rows,
+                                  int32_t R, float scale, float* map, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (R < 1) return fail(VEDA_ERR_INVALID_ARG, "R must be >= 1 (got %d)", R);
+  if (!qp || !kp || !rows || !map || !workspace) return fail(VEDA_ERR_INVALID_ARG, "NULL tensor argument");
+  if (!aligned16(qp) || !aligned16(kp) || !aligned16(map) || !aligned16(rows))
+    return fail(VEDA_ERR_INVALID_ARG, "tensor arguments must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(VEDA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (workspace_bytes < map_ws_bytes(G, R))
+    return fail(VEDA_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, map_ws_bytes(G, R));
+  if ((long long)G.B * G.heads * R >= (1LL << 31)) return fail(VEDA_ERR_INVALID_ARG, "B*heads*R too large");
+  if (!(std::isfinite(scale))) return fail(VEDA_ERR_INVALID_ARG, "scale must be finite");
+  CUtensorMap tq, tk;
+  if ((s = encode_tile_major(G, qp, &tq)) != VEDA_OK || (s = encode_tile_major(G, kp, &tk)) != VEDA_OK) return s;
+  MapArgs a;
+  a.rows = rows;
+  a.R = R;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)G.d);
+  a.scale_log2 = sc * 1.4426950408889634f;
+  a.rowmax = static_cast<float*>(workspace);
+  a.lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + map_rowmax_bytes(G, R));
+  a.map = map;
+  a.timeout_ns = g_timeout_ns;
+  cudaError_t e = launch_tile_map(G, tq, tk, a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "veda_tile_map_maxpool");
+  return ok();
+}
+
+veda_status veda_sync_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "veda_sync_status: stream synchronize");
+  int word = 0;
+  e = cudaMemcpyFromSymbol(&word, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "veda_sync_status: read device error word");
+  if (word != kErrNone) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+    return fail(VEDA_ERR_TIMEOUT, "a kernel gave up on a bounded wait (device error word %d)", word);
+  }
+  return ok();
+}
+
+veda_status veda_set_wait_timeout_ns(uint64_t ns) {
+  if (ns < 1000ull || ns > 60000000000ull) return fail(VEDA_ERR_INVALID_ARG, "timeout must be in [1 us, 60 s]");
+  g_timeout_ns = ns;
+  return ok();
+}
+
+veda_status veda_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
+  if (timeout_ns < 1000ull || timeout_ns > 10000000000ull)
+    return fail(VEDA_ERR_INVALID_ARG, "timeout must be in [1 us, 10 s]");
+  cudaError_t e = launch_timeout_selftest(timeout_ns, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "veda_selftest_wait_timeout");
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+"""The whole inference path as one call sequence over the C ABI.
+
+``VedaAttention`` owns the device buffers (torch allocations: memory
+plumbing only) and enqueues, on one CUDA stream,
+
+    veda_tile_permute(Q), (K), (V) -> veda_tripool(Qp), (Kp)
+    -> veda_tile_score_topk -> veda_tile_sparse_attn -> veda_tile_unpermute
+
+which is the per-layer path of Veda's tile-sparse attention (technical
+summary, sections 2.1-2.3).  Every step runs in the library's kernels.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import binding as B
+
+
+class VedaAttention:
+    def __init__(self, problem: B.Problem, mlp_q, mlp_k, keep_ratio: float, device="cuda",
+                 want_probs: bool = False, want_lse: bool = False):
+        """mlp_q / mlp_k: (w1, b1, w2, b2) fp32 tensors on ``device`` (may be the same)."""
+        self.p = problem
+        self.keep = float(keep_ratio)
+        self.k_per_head, self.k_max = problem.keep_count(self.keep)
+        self._wq = tuple(mlp_q)
+        self._wk = tuple(mlp_k)
+        self.mlp_q = B.make_mlp(*self._wq)
+        self.mlp_k = B.make_mlp(*self._wk)
+        p = problem
+        ts = p.tile_shape()
+        self.qp = torch.empty(ts, dtype=torch.bfloat16, device=device)
+        self.kp = torch.empty(ts, dtype=torch.bfloat16, device=device)
+        self.vp = torch.empty(ts, dtype=torch.bfloat16, device=device)
+        self.op = torch.empty(ts, dtype=torch.bfloat16, device=device)
+        self.desc_q = torch.empty((p.B, p.heads, p.nt_max, 3 * p.d), dtype=torch.float32, device=device)
+        self.desc_k = torch.empty_like(self.desc_q)
+        self.idx = torch.empty((p.B, p.heads, p.nt_max, self.k_max), dtype=torch.int32, device=device)
+        self.probs = (torch.empty((p.B, p.heads, p.nt_max, p.nt_max), dtype=torch.float32, device=device)
+                      if want_probs else None)
+        self.lse = (torch.empty((p.B, p.heads, p.nt_max * p.S), dtype=torch.float32, device=device)
+                    if want_lse else None)
+        ws = B.veda_score_topk_workspace(p, self.mlp_q.e)
+        self.workspace = torch.empty(ws // 4 + 64, dtype=torch.float32, device=device)
+
+    def select(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None) -> torch.Tensor:
+        """Permute, pool and score; returns the selected tile indices."""
+        p = self.p
+        B.veda_tile_permute(p, q, self.qp, stream)
+        B.veda_tile_permute(p, k, self.kp, stream)
+        B.veda_tile_permute(p, v, self.vp, stream)
+        B.veda_tripool(p, self.qp, self.desc_q, stream)
+        B.veda_tripool(p, self.kp, self.desc_k, stream)
+        B.veda_tile_score_topk(p, self.desc_q, self.desc_k, self.mlp_q, self.mlp_k, self.keep, self.idx, self.probs,
+                               self.workspace, stream)
+        return self.idx
+
+    def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+        """Grid-order bf16 Q, K, V [B, heads, N, d] -> grid-order output of the same shape."""
+        p = self.p
+        if out is None:
+            out = torch.empty(p.grid_shape(), dtype=torch.bfloat16, device=q.device)
+        self.select(q, k, v, stream)
+        B.veda_tile_sparse_attn(p, self.qp, self.kp, self.vp, self.idx, self.op, self.lse, 0.0, stream)
+        B.veda_tile_unpermute(p, self.op, out, stream)
+        return out
