@@ -159,12 +159,10 @@ def run_ours(args, world, rank, local):
             att(qd, kd, vd, out)
             return
         ev[0].record()
-        V.veda_tile_permute(p, qd, att.qp)
-        V.veda_tile_permute(p, kd, att.kp)
-        V.veda_tile_permute(p, vd, att.vp)
+        V.veda_tile_permute_tripool(p, qd, att.qp, att.desc_q)
+        V.veda_tile_permute_tripool(p, kd, att.kp, att.desc_k)
         ev[1].record()
-        V.veda_tripool(p, att.qp, att.desc_q)
-        V.veda_tripool(p, att.kp, att.desc_k)
+        V.veda_tile_permute(p, vd, att.vp)
         ev[2].record()
         V.veda_tile_score_topk(p, att.desc_q, att.desc_k, att.mlp_q, att.mlp_k, att.keep, att.idx, None,
                                att.workspace)
@@ -197,9 +195,9 @@ def run_ours(args, world, rank, local):
     V.veda_sync_status()
     ms_total = max_over_ranks(t0.elapsed_time(t1), world)
     ms_step = ms_total / args.steps
-    stage = {"permute": [], "tripool": [], "score_topk": [], "attention": [], "unpermute": []}
+    stage = {"permute_tripool_qk": [], "permute_v": [], "score_topk": [], "attention": [], "unpermute": []}
     for ev in evs:
-        for name, a, b in (("permute", 0, 1), ("tripool", 1, 2), ("score_topk", 2, 3), ("attention", 3, 4),
+        for name, a, b in (("permute_tripool_qk", 0, 1), ("permute_v", 1, 2), ("score_topk", 2, 3), ("attention", 3, 4),
                            ("unpermute", 4, 5)):
             stage[name].append(ev[a].elapsed_time(ev[b]))
     stage_ms = {k: float(np.mean(v)) for k, v in stage.items()}
@@ -250,7 +248,7 @@ def run_ours(args, world, rank, local):
                       "l2": "inputs (3 x %.0f MB) larger than L2; no flush" % (q.numel() * 2 / 1e6)},
            "ms_per_layer": ms_step, "stage_ms": stage_ms, "attn_tflops": achieved,
            "pct_of_bf16_peak": 100.0 * achieved / peaks["bf16_tflops"],
-           "roofline": roofline, "gpu_launches": 9 * args.steps, "clocks": clk, "e2e": e2e}
+           "roofline": roofline, "gpu_launches": 7 * args.steps, "clocks": clk, "e2e": e2e}
     return res, (w, p, ks, flops)
 
 

@@ -73,7 +73,8 @@ typedef struct {
 /* Per-head two-layer estimator (section 2.1, "head-specific MLP
  * projections"): phi = W2 relu(W1 desc + b1) + b2.  DEVICE fp32 pointers:
  * w1 [heads, hidden, 3d], b1 [heads, hidden], w2 [heads, e, hidden],
- * b2 [heads, e], all row-major.  hidden <= 512, e <= 128, e % 4 == 0. */
+ * b2 [heads, e], all row-major.  hidden a multiple of 4 in [4, 512];
+ * e in {16, 32, 64, 128}. */
 typedef struct {
   const float* w1;
   const float* b1;
@@ -117,6 +118,14 @@ veda_status veda_tile_unpermute(const veda_problem* p, const void* xp, void* x, 
  * desc[.., j, 0:d] = mean, [d:2d] = max, [2d:3d] = min over the token slots of
  * tile j (pad slots excluded); rows j >= NT_h are zero. */
 veda_status veda_tripool(const veda_problem* p, const void* xp, float* desc, void* stream);
+
+/* veda_tile_permute and veda_tripool in one pass over x (the pages' future
+ * work names "tighter kernel fusion", section 5): xp as veda_tile_permute
+ * writes it and desc as veda_tripool would compute it from xp, with x read
+ * from HBM once.  Arguments as in the two calls; x, xp and desc must not
+ * overlap. */
+veda_status veda_tile_permute_tripool(const veda_problem* p, const void* x, void* xp, float* desc,
+                                      void* stream);
 
 /* ---------------------------------------------------------------- steps 3-4: estimator + top-k */
 

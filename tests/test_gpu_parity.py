@@ -84,6 +84,25 @@ def test_tripool(run):
         np.testing.assert_allclose(g[..., :d], ref[..., :d], rtol=MEAN_REL, atol=1e-6)
 
 
+def test_tripool_standalone_matches_fused(V, run):
+    """veda_tripool on the permuted tensor gives the fused permute+TripPool descriptor."""
+    p, d = run.p, run.w.d
+    desc = torch.full_like(run.att.desc_k, float("nan"))
+    V.veda_tripool(p, run.att.kp, desc)
+    V.veda_sync_status()
+    g, ref = f64(desc), run.ora["desc_k"]
+    np.testing.assert_array_equal(g[..., d:], ref[..., d:])
+    np.testing.assert_allclose(g[..., :d], ref[..., :d], rtol=MEAN_REL, atol=1e-6)
+    assert torch.equal(desc, run.att.desc_k)
+
+
+def test_permute_alone_matches_fused(V, run):
+    qp = torch.empty_like(run.att.qp)
+    V.veda_tile_permute(run.p, run.q.cuda(), qp)
+    torch.cuda.synchronize()
+    assert torch.equal(qp, run.att.qp)
+
+
 def test_score_topk(run):
     nts = run.p.nt_per_head
     ks, _ = run.p.keep_count(run.w.keep)

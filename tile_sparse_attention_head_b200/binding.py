@@ -56,6 +56,7 @@ _SIG = {
     "veda_keep_count": [_P, ctypes.c_float, _I32P, _I32P],
     "veda_tile_permute": [_P, _V, _V, _V],
     "veda_tile_unpermute": [_P, _V, _V, _V],
+    "veda_tile_permute_tripool": [_P, _V, _V, _V, _V],
     "veda_tripool": [_P, _V, _V, _V],
     "veda_score_topk_workspace": [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)],
     "veda_tile_score_topk": [_P, _V, _V, ctypes.POINTER(veda_mlp), ctypes.POINTER(veda_mlp), ctypes.c_float, _V,
@@ -159,6 +160,15 @@ def veda_tile_permute(p: Problem, x: torch.Tensor, xp: torch.Tensor, stream=None
     _check(LIB.veda_tile_permute(p.ref, _ptr(x, "x", torch.bfloat16, p.grid_shape()),
                                  _ptr(xp, "xp", torch.bfloat16, p.tile_shape()), _stream(stream)),
            "veda_tile_permute")
+    return xp
+
+
+def veda_tile_permute_tripool(p: Problem, x: torch.Tensor, xp: torch.Tensor, desc: torch.Tensor,
+                              stream=None) -> torch.Tensor:
+    _check(LIB.veda_tile_permute_tripool(p.ref, _ptr(x, "x", torch.bfloat16, p.grid_shape()),
+                                         _ptr(xp, "xp", torch.bfloat16, p.tile_shape()),
+                                         _ptr(desc, "desc", torch.float32, (p.B, p.heads, p.nt_max, 3 * p.d)),
+                                         _stream(stream)), "veda_tile_permute_tripool")
     return xp
 
 

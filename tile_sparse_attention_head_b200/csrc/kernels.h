@@ -45,9 +45,12 @@ struct MapArgs {
 
 cudaError_t launch_permute(const Geometry& G, const void* x, void* xp, cudaStream_t s, int sms);
 cudaError_t launch_unpermute(const Geometry& G, const void* xp, void* x, cudaStream_t s, int sms);
+cudaError_t launch_permute_tripool(const Geometry& G, const void* x, void* xp, float* desc, cudaStream_t s);
 cudaError_t launch_tripool(const Geometry& G, const void* xp, float* desc, cudaStream_t s);
 
-size_t estimator_smem_bytes(int d, int hidden);
+size_t estimator_smem_bytes(int d, int hidden, int e);
+cudaError_t launch_estimator(const Geometry& G, const float* dq, const float* dk, const EstimatorWeights& wq,
+                             const EstimatorWeights& wk, int hidden, int e, float* phi, cudaStream_t s);
 void score_topk_config(int ntmax, int e, int* qb, int* ntpad, size_t* smem);
 cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const float* desc_k,
                               const EstimatorWeights& wq, const EstimatorWeights& wk, int hidden,

@@ -2,97 +2,32 @@
 // tiling", section 2.2 of the Veda summary) and the TripPool descriptor
 // (section 2.1: channel-wise mean, max and min of each tile, concatenated).
 //
-// All three move 16-byte vectors (8 bf16 channels) per thread so every warp
-// touches whole 128-byte lines; the permutations are output-driven so each
-// output row is written exactly once (pad slots as zeros).
+// Layout of the work: one CTA per (b, h, tile) for the permutation, one per
+// (b, h, 128 grid rows) for the inverse.  The index arithmetic (divisions by
+// the tiling factors) is done once per row by one thread into shared memory;
+// the copy phase then moves 16-byte vectors (8 bf16 channels) with every
+// thread keeping several independent loads in flight, so whole 128-byte lines
+// move per warp.  The permutation can also produce the TripPool descriptor
+// of the tile it is writing (fused: the tile is read from HBM once).
 #include "veda_common.cuh"
 #include "kernels.h"
 
 namespace veda {
 
-// Xp[b,h, j*S + l, :] = X[b,h, n(j,l), :], zeros for pad slots and j >= NT_h.
-// One thread per 16-byte chunk of an output row; grid-stride.
-__global__ void __launch_bounds__(256) permute_kernel(const __grid_constant__ Geometry G,
-                                                      const uint4* __restrict__ x,
-                                                      uint4* __restrict__ xp) {
-  const int cpr = G.d >> 3;  // 16-byte chunks per row
-  const long long rows_per_head = (long long)G.ntmax * G.S;
-  const long long total = (long long)G.B * G.heads * rows_per_head * cpr;
-  for (long long c = blockIdx.x * (long long)blockDim.x + threadIdx.x; c < total;
-       c += (long long)gridDim.x * blockDim.x) {
-    const int chunk = (int)(c % cpr);
-    const long long row = c / cpr;
-    const int r = (int)(row % rows_per_head);
-    const long long bh = row / rows_per_head;
-    const int h = (int)(bh % G.heads);
-    const HeadGeom& hg = G.g[h];
-    const int j = r / G.S, l = r % G.S;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (j < hg.nt) {
-      const int n = slot_to_grid(G, hg, j, l);
-      if (n >= 0) v = __ldg(x + ((bh * G.N + n) * cpr + chunk));
-    }
-    xp[c] = v;
-  }
-}
+constexpr int kPermThreads = 256;
 
-// X[b,h, n, :] = Xp[b,h, pos_h(n), :].  One thread per 16-byte chunk of a grid row.
-__global__ void __launch_bounds__(256) unpermute_kernel(const __grid_constant__ Geometry G,
-                                                        const uint4* __restrict__ xp,
-                                                        uint4* __restrict__ x) {
-  const int cpr = G.d >> 3;
-  const long long rows_per_head_p = (long long)G.ntmax * G.S;
-  const long long total = (long long)G.B * G.heads * G.N * cpr;
-  for (long long c = blockIdx.x * (long long)blockDim.x + threadIdx.x; c < total;
-       c += (long long)gridDim.x * blockDim.x) {
-    const int chunk = (int)(c % cpr);
-    const long long row = c / cpr;
-    const int n = (int)(row % G.N);
-    const long long bh = row / G.N;
-    const int h = (int)(bh % G.heads);
-    const int pos = grid_to_slot(G, G.g[h], n);
-    x[c] = __ldg(xp + ((bh * rows_per_head_p + pos) * cpr + chunk));
-  }
-}
-
-// TripPool: one warp per (b, h, tile).  Lanes split a tile row into 16-byte
-// chunks (8 channels); with d = 128 a warp covers 2 rows per step, with
-// d = 64 four.  Each lane keeps fp32 sum / max / min of its 8 channels over
-// the token slots it visits; lanes sharing a chunk are then combined by
-// shuffles.  desc = [mean || max || min], fp32.
-template <int D>
-__global__ void __launch_bounds__(256) tripool_kernel(const __grid_constant__ Geometry G,
-                                                      const uint4* __restrict__ xp,
-                                                      float* __restrict__ desc) {
-  constexpr int CPR = D / 8;          // chunks per row
-  constexpr int RPS = 32 / CPR;       // rows per warp step
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const long long ntiles = (long long)G.B * G.heads * G.ntmax;
-  if (warp >= ntiles) return;
-  const int j = (int)(warp % G.ntmax);
-  const long long bh = warp / G.ntmax;
-  const int h = (int)(bh % G.heads);
-  const HeadGeom& hg = G.g[h];
-  float* out = desc + (long long)warp * 3 * D;
-  const int chunk = lane % CPR;
-  if (j >= hg.nt) {
-    for (int c = lane; c < 3 * D; c += 32) out[c] = 0.f;
-    return;
-  }
+// Per-thread running statistics of 8 channels.
+struct Stats8 {
   float sum[8], mx[8], mn[8];
+  __device__ __forceinline__ void init() {
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    sum[k] = 0.f;
-    mx[k] = -INFINITY;
-    mn[k] = INFINITY;
+    for (int k = 0; k < 8; ++k) {
+      sum[k] = 0.f;
+      mx[k] = -INFINITY;
+      mn[k] = INFINITY;
+    }
   }
-  const uint4* base = xp + ((bh * G.ntmax + j) * (long long)G.S) * CPR;
-  const int full = (tile_token_count(G, hg, j) == G.S);
-  for (int r0 = 0; r0 < G.S; r0 += RPS) {
-    const int l = r0 + lane / CPR;
-    if (!full && slot_to_grid(G, hg, j, l) < 0) continue;
-    const uint4 v = __ldg(base + (long long)l * CPR + chunk);
+  __device__ __forceinline__ void add(const uint4& v) {
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -105,56 +40,189 @@ __global__ void __launch_bounds__(256) tripool_kernel(const __grid_constant__ Ge
       mn[2 * k + 1] = fminf(mn[2 * k + 1], f.y);
     }
   }
+};
+
+// Combines the per-thread statistics of all threads that own the same
+// 16-byte chunk of a row (threads tid, tid + CPR, ...) and writes
+// desc = [mean || max || min] for the tile.  `red` holds 3 * 256 * 8 floats.
+template <int D>
+__device__ __forceinline__ void tripool_reduce_store(const Stats8& st, float* red, int count, float* out) {
+  constexpr int CPR = D / 8;
+  constexpr int GROUPS = kPermThreads / CPR;
+  const int tid = threadIdx.x;
 #pragma unroll
-  for (int off = CPR; off < 32; off <<= 1) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      sum[k] += __shfl_xor_sync(0xffffffffu, sum[k], off);
-      mx[k] = fmaxf(mx[k], __shfl_xor_sync(0xffffffffu, mx[k], off));
-      mn[k] = fminf(mn[k], __shfl_xor_sync(0xffffffffu, mn[k], off));
+  for (int k = 0; k < 8; ++k) {
+    red[(0 * kPermThreads + tid) * 8 + k] = st.sum[k];
+    red[(1 * kPermThreads + tid) * 8 + k] = st.mx[k];
+    red[(2 * kPermThreads + tid) * 8 + k] = st.mn[k];
+  }
+  __syncthreads();
+  // Thread c (< D) finishes channel c: chunk c/8, lane-in-chunk c%8.
+  for (int c = tid; c < D; c += kPermThreads) {
+    const int chunk = c >> 3, k = c & 7;
+    float s = 0.f, mx = -INFINITY, mn = INFINITY;
+#pragma unroll 4
+    for (int g = 0; g < GROUPS; ++g) {
+      const int t = g * CPR + chunk;
+      s += red[(0 * kPermThreads + t) * 8 + k];
+      mx = fmaxf(mx, red[(1 * kPermThreads + t) * 8 + k]);
+      mn = fminf(mn, red[(2 * kPermThreads + t) * 8 + k]);
     }
-  }
-  if (lane < CPR) {
-    const float inv = 1.0f / (float)tile_token_count(G, hg, j);
-    float4* o_mean = reinterpret_cast<float4*>(out + chunk * 8);
-    float4* o_max = reinterpret_cast<float4*>(out + D + chunk * 8);
-    float4* o_min = reinterpret_cast<float4*>(out + 2 * D + chunk * 8);
-    o_mean[0] = make_float4(sum[0] * inv, sum[1] * inv, sum[2] * inv, sum[3] * inv);
-    o_mean[1] = make_float4(sum[4] * inv, sum[5] * inv, sum[6] * inv, sum[7] * inv);
-    o_max[0] = make_float4(mx[0], mx[1], mx[2], mx[3]);
-    o_max[1] = make_float4(mx[4], mx[5], mx[6], mx[7]);
-    o_min[0] = make_float4(mn[0], mn[1], mn[2], mn[3]);
-    o_min[1] = make_float4(mn[4], mn[5], mn[6], mn[7]);
+    out[c] = s / (float)count;
+    out[D + c] = mx;
+    out[2 * D + c] = mn;
   }
 }
 
-static int grid_for(long long work, int threads, int sms) {
-  long long blocks = (work + threads - 1) / threads;
-  const long long cap = (long long)sms * 16;
-  if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
-  return (int)blocks;
+// grid: (NT_max, B*heads).  Writes all S rows of tile j of head h (zeros for
+// pad slots and tiles j >= NT_h); with POOL also desc[b, h, j, :].
+template <int D, int S, bool POOL>
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(const __grid_constant__ Geometry G,
+                                                               const uint4* __restrict__ x,
+                                                               uint4* __restrict__ xp,
+                                                               float* __restrict__ desc) {
+  constexpr int CPR = D / 8;                        // 16-byte chunks per row
+  constexpr int RPP = kPermThreads / CPR;           // rows per pass
+  constexpr int PASSES = S / RPP;
+  __shared__ int s_src[S];
+  __shared__ float s_red[POOL ? 3 * kPermThreads * 8 : 1];
+  const int j = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int h = bh % G.heads;
+  const HeadGeom& hg = G.g[h];
+  const int tid = threadIdx.x;
+  const bool live = j < hg.nt;
+  if (tid < S) s_src[tid] = live ? slot_to_grid(G, hg, j, tid) : -1;
+  __syncthreads();
+
+  const uint4* xb = x + (size_t)bh * G.N * CPR;
+  uint4* xo = xp + ((size_t)bh * G.ntmax + j) * (size_t)S * CPR;
+  const int chunk = tid % CPR, r0 = tid / CPR;
+  uint4 v[PASSES];
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p) {
+    const int n = s_src[r0 + p * RPP];
+    v[p] = (n >= 0) ? __ldg(xb + (size_t)n * CPR + chunk) : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p) xo[(size_t)(r0 + p * RPP) * CPR + chunk] = v[p];
+
+  if constexpr (POOL) {
+    float* out = desc + ((size_t)bh * G.ntmax + j) * 3 * D;
+    if (!live) {
+      for (int c = tid; c < 3 * D; c += kPermThreads) out[c] = 0.f;
+      return;
+    }
+    Stats8 st;
+    st.init();
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p)
+      if (s_src[r0 + p * RPP] >= 0) st.add(v[p]);
+    tripool_reduce_store<D>(st, s_red, tile_token_count(G, hg, j), out);
+  }
 }
 
-cudaError_t launch_permute(const Geometry& G, const void* x, void* xp, cudaStream_t s, int sms) {
-  const long long work = (long long)G.B * G.heads * G.ntmax * G.S * (G.d / 8);
-  permute_kernel<<<grid_for(work, 256, sms), 256, 0, s>>>(G, (const uint4*)x, (uint4*)xp);
+// TripPool alone, from an already permuted tensor.  grid: (NT_max, B*heads).
+template <int D, int S>
+__global__ void __launch_bounds__(kPermThreads) tripool_kernel(const __grid_constant__ Geometry G,
+                                                               const uint4* __restrict__ xp,
+                                                               float* __restrict__ desc) {
+  constexpr int CPR = D / 8;
+  constexpr int RPP = kPermThreads / CPR;
+  constexpr int PASSES = S / RPP;
+  __shared__ unsigned char s_valid[S];
+  __shared__ float s_red[3 * kPermThreads * 8];
+  const int j = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int h = bh % G.heads;
+  const HeadGeom& hg = G.g[h];
+  const int tid = threadIdx.x;
+  float* out = desc + ((size_t)bh * G.ntmax + j) * 3 * D;
+  if (j >= hg.nt) {
+    for (int c = tid; c < 3 * D; c += kPermThreads) out[c] = 0.f;
+    return;
+  }
+  if (tid < S) s_valid[tid] = slot_to_grid(G, hg, j, tid) >= 0;
+  __syncthreads();
+  const uint4* xi = xp + ((size_t)bh * G.ntmax + j) * (size_t)S * CPR;
+  const int chunk = tid % CPR, r0 = tid / CPR;
+  uint4 v[PASSES];
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p) v[p] = __ldg(xi + (size_t)(r0 + p * RPP) * CPR + chunk);
+  Stats8 st;
+  st.init();
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p)
+    if (s_valid[r0 + p * RPP]) st.add(v[p]);
+  tripool_reduce_store<D>(st, s_red, tile_token_count(G, hg, j), out);
+}
+
+// X[b,h, n, :] = Xp[b,h, pos_h(n), :].  grid: (ceil(N / 128), B*heads).
+template <int D>
+__global__ void __launch_bounds__(kPermThreads) unpermute_kernel(const __grid_constant__ Geometry G,
+                                                                 const uint4* __restrict__ xp,
+                                                                 uint4* __restrict__ x) {
+  constexpr int CPR = D / 8;
+  constexpr int ROWS = 128;
+  constexpr int RPP = kPermThreads / CPR;
+  constexpr int PASSES = ROWS / RPP;
+  __shared__ int s_pos[ROWS];
+  const int bh = blockIdx.y;
+  const int h = bh % G.heads;
+  const int n0 = blockIdx.x * ROWS;
+  const int tid = threadIdx.x;
+  if (tid < ROWS) s_pos[tid] = (n0 + tid < G.N) ? grid_to_slot(G, G.g[h], n0 + tid) : -1;
+  __syncthreads();
+  const uint4* xi = xp + (size_t)bh * G.ntmax * G.S * CPR;
+  uint4* xo = x + ((size_t)bh * G.N + n0) * CPR;
+  const int chunk = tid % CPR, r0 = tid / CPR;
+  uint4 v[PASSES];
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p) {
+    const int pos = s_pos[r0 + p * RPP];
+    if (pos >= 0) v[p] = __ldg(xi + (size_t)pos * CPR + chunk);
+  }
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p)
+    if (s_pos[r0 + p * RPP] >= 0) xo[(size_t)(r0 + p * RPP) * CPR + chunk] = v[p];
+}
+
+template <bool POOL>
+static cudaError_t launch_permute_t(const Geometry& G, const void* x, void* xp, float* desc, cudaStream_t s) {
+  dim3 grid(G.ntmax, G.B * G.heads);
+  const uint4* xi = (const uint4*)x;
+  uint4* xo = (uint4*)xp;
+  if (G.d == 128 && G.S == 128) permute_kernel<128, 128, POOL><<<grid, kPermThreads, 0, s>>>(G, xi, xo, desc);
+  else if (G.d == 128) permute_kernel<128, 64, POOL><<<grid, kPermThreads, 0, s>>>(G, xi, xo, desc);
+  else if (G.S == 128) permute_kernel<64, 128, POOL><<<grid, kPermThreads, 0, s>>>(G, xi, xo, desc);
+  else permute_kernel<64, 64, POOL><<<grid, kPermThreads, 0, s>>>(G, xi, xo, desc);
   return cudaGetLastError();
 }
 
+cudaError_t launch_permute(const Geometry& G, const void* x, void* xp, cudaStream_t s, int sms) {
+  (void)sms;
+  return launch_permute_t<false>(G, x, xp, nullptr, s);
+}
+
+cudaError_t launch_permute_tripool(const Geometry& G, const void* x, void* xp, float* desc, cudaStream_t s) {
+  return launch_permute_t<true>(G, x, xp, desc, s);
+}
+
 cudaError_t launch_unpermute(const Geometry& G, const void* xp, void* x, cudaStream_t s, int sms) {
-  const long long work = (long long)G.B * G.heads * G.N * (G.d / 8);
-  unpermute_kernel<<<grid_for(work, 256, sms), 256, 0, s>>>(G, (const uint4*)xp, (uint4*)x);
+  (void)sms;
+  dim3 grid((G.N + 127) / 128, G.B * G.heads);
+  if (G.d == 128) unpermute_kernel<128><<<grid, kPermThreads, 0, s>>>(G, (const uint4*)xp, (uint4*)x);
+  else unpermute_kernel<64><<<grid, kPermThreads, 0, s>>>(G, (const uint4*)xp, (uint4*)x);
   return cudaGetLastError();
 }
 
 cudaError_t launch_tripool(const Geometry& G, const void* xp, float* desc, cudaStream_t s) {
-  const long long warps = (long long)G.B * G.heads * G.ntmax;
-  const int blocks = (int)((warps * 32 + 255) / 256);
-  if (G.d == 128)
-    tripool_kernel<128><<<blocks, 256, 0, s>>>(G, (const uint4*)xp, desc);
-  else
-    tripool_kernel<64><<<blocks, 256, 0, s>>>(G, (const uint4*)xp, desc);
+  dim3 grid(G.ntmax, G.B * G.heads);
+  const uint4* xi = (const uint4*)xp;
+  if (G.d == 128 && G.S == 128) tripool_kernel<128, 128><<<grid, kPermThreads, 0, s>>>(G, xi, desc);
+  else if (G.d == 128) tripool_kernel<128, 64><<<grid, kPermThreads, 0, s>>>(G, xi, desc);
+  else if (G.S == 128) tripool_kernel<64, 128><<<grid, kPermThreads, 0, s>>>(G, xi, desc);
+  else tripool_kernel<64, 64><<<grid, kPermThreads, 0, s>>>(G, xi, desc);
   return cudaGetLastError();
 }
 

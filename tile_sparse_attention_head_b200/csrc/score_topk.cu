@@ -14,97 +14,9 @@
 // evaluation on genuine near-ties.
 #include "veda_common.cuh"
 #include "kernels.h"
+#include "estimator.cu"
 
 namespace veda {
-
-constexpr int kEstTiles = 32;     // tiles per estimator CTA
-constexpr int kEstThreads = 256;
-constexpr int kEstChunk = 32;     // input channels staged per step
-
-// grid: (ceil(NT_max / 32), B*heads, 2)  z = 0: Q descriptors, z = 1: K.
-__global__ void __launch_bounds__(kEstThreads)
-    estimator_kernel(const __grid_constant__ Geometry G, const float* __restrict__ desc_q,
-                     const float* __restrict__ desc_k, EstimatorWeights wq, EstimatorWeights wk,
-                     int hidden, int e, float* __restrict__ phi) {
-  extern __shared__ float sm[];
-  const int in_dim = 3 * G.d;
-  const int which = blockIdx.z;
-  const int bh = blockIdx.y;
-  const int h = bh % G.heads;
-  const int nt = G.g[h].nt;
-  const int j0 = blockIdx.x * kEstTiles;
-  if (j0 >= nt) return;
-  const int ntile = min(kEstTiles, nt - j0);
-  const EstimatorWeights& w = which ? wk : wq;
-  const float* desc = (which ? desc_k : desc_q) + ((long long)bh * G.ntmax + j0) * in_dim;
-  const float* W1 = w.w1 + (long long)h * hidden * in_dim;
-  const float* B1 = w.b1 + (long long)h * hidden;
-  const float* W2 = w.w2 + (long long)h * e * hidden;
-  const float* B2 = w.b2 + (long long)h * e;
-
-  float* s_desc = sm;                                  // [32][in_dim]
-  float* s_w1 = s_desc + kEstTiles * in_dim;           // [hidden][33]
-  float* s_hid = s_w1 + hidden * (kEstChunk + 1);      // [32][hidden]
-  const int tid = threadIdx.x;
-
-  for (int i = tid; i < kEstTiles * in_dim; i += kEstThreads) {
-    const int t = i / in_dim;
-    s_desc[i] = (t < ntile) ? desc[i] : 0.f;
-  }
-
-  // Layer 1: each thread owns hidden units u = tid, tid + 256 (hidden <= 512).
-  float acc[2][kEstTiles];
-#pragma unroll
-  for (int a = 0; a < 2; ++a)
-#pragma unroll
-    for (int t = 0; t < kEstTiles; ++t) acc[a][t] = 0.f;
-
-  for (int c0 = 0; c0 < in_dim; c0 += kEstChunk) {
-    __syncthreads();
-    for (int i = tid; i < hidden * kEstChunk; i += kEstThreads) {
-      const int u = i / kEstChunk, c = i % kEstChunk;
-      s_w1[u * (kEstChunk + 1) + c] = W1[(long long)u * in_dim + c0 + c];
-    }
-    __syncthreads();
-#pragma unroll
-    for (int a = 0; a < 2; ++a) {
-      const int u = tid + a * kEstThreads;
-      if (u < hidden) {
-        for (int c = 0; c < kEstChunk; ++c) {
-          const float wv = s_w1[u * (kEstChunk + 1) + c];
-#pragma unroll
-          for (int t = 0; t < kEstTiles; ++t) acc[a][t] = fmaf(s_desc[t * in_dim + c0 + c], wv, acc[a][t]);
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int a = 0; a < 2; ++a) {
-    const int u = tid + a * kEstThreads;
-    if (u < hidden) {
-      const float bb = B1[u];
-#pragma unroll
-      for (int t = 0; t < kEstTiles; ++t) s_hid[t * hidden + u] = fmaxf(acc[a][t] + bb, 0.f);
-    }
-  }
-  __syncthreads();
-
-  // Layer 2: kEstTiles * e outputs spread over the block.
-  float* out = phi + (((long long)which * G.B * G.heads + bh) * G.ntmax + j0) * e;
-  for (int i = tid; i < ntile * e; i += kEstThreads) {
-    const int t = i / e, o = i % e;
-    const float* w2row = W2 + (long long)o * hidden;
-    const float* hrow = s_hid + t * hidden;
-    float acc2 = 0.f;
-    for (int k = 0; k < hidden; ++k) acc2 = fmaf(hrow[k], __ldg(w2row + k), acc2);
-    out[(long long)t * e + o] = acc2 + B2[o];
-  }
-}
-
-size_t estimator_smem_bytes(int d, int hidden) {
-  return sizeof(float) * ((size_t)kEstTiles * 3 * d + (size_t)hidden * (kEstChunk + 1) +
-                          (size_t)kEstTiles * hidden);
-}
 
 // Order-preserving map fp32 -> uint32 (larger float <-> larger key).
 __device__ __forceinline__ uint32_t float_key(float f) {
@@ -278,13 +190,8 @@ __global__ void __launch_bounds__(kScoreThreads)
 cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const float* desc_k,
                               const EstimatorWeights& wq, const EstimatorWeights& wk, int hidden,
                               int e, float* phi, const TopkArgs& args, cudaStream_t s) {
-  const size_t est_smem = estimator_smem_bytes(G.d, hidden);
-  cudaError_t err = cudaFuncSetAttribute(estimator_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)est_smem);
+  cudaError_t err = launch_estimator(G, desc_q, desc_k, wq, wk, hidden, e, phi, s);
   if (err != cudaSuccess) return err;
-  dim3 g1((G.ntmax + kEstTiles - 1) / kEstTiles, G.B * G.heads, 2);
-  estimator_kernel<<<g1, kEstThreads, est_smem, s>>>(G, desc_q, desc_k, wq, wk, hidden, e, phi);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
 
   int qb, ntpad;
   size_t smem;

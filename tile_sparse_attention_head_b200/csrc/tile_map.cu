@@ -24,6 +24,11 @@
 
 namespace veda {
 
+// Pass 1 is exponential-bound (Q K^T only); one exponential in
+// kMapPolyEvery runs on the FMA pipe (exp2_fma), the rest on the
+// special-function unit.
+constexpr int kMapPolyEvery = 3;
+
 template <int D, int BN>
 struct MapCfg {
   static constexpr int BM = 128;
@@ -199,15 +204,27 @@ __global__ void __launch_bounds__(192, 1)
         for (int c = 0; c < BN; ++c)
           if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
       }
-      float mt = -INFINITY;
+      float m8[8];
 #pragma unroll
-      for (int c = 0; c < BN; ++c) mt = fmaxf(mt, s[c]);
+      for (int q = 0; q < 8; ++q) m8[q] = s[q];
+#pragma unroll
+      for (int c = 8; c < BN; c += 8)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) m8[q] = fmaxf(m8[q], s[c + q]);
+      float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       mt *= sl2;
       if (row < S) rm[(long long)t * S] = mt;
       const float m_new = fmaxf(m_run, mt);
-      float rs = 0.f;
+      float r8[8];
 #pragma unroll
-      for (int c = 0; c < BN; ++c) rs += fast_exp2(fmaf(s[c], sl2, -m_new));
+      for (int q = 0; q < 8; ++q) r8[q] = 0.f;
+#pragma unroll
+      for (int c = 0; c < BN; ++c) {
+        const float x = fmaf(s[c], sl2, -m_new);
+        r8[c & 7] += (c % kMapPolyEvery == kMapPolyEvery - 1) ? exp2_fma(x) : fast_exp2(x);
+      }
+      const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       l_run = l_run * fast_exp2(m_run - m_new) + rs;
       m_run = m_new;
     }

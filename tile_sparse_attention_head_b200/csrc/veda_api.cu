@@ -94,6 +94,7 @@ veda_status make_geometry(const veda_problem* p, Geometry* G) {
   if (rows >= (1LL << 31)) return fail(VEDA_ERR_INVALID_ARG, "B*heads*NT_max*S = %lld rows exceeds 2^31", rows);
   if ((long long)p->B * p->heads * N >= (1LL << 31))
     return fail(VEDA_ERR_INVALID_ARG, "B*heads*N exceeds 2^31 rows");
+  if ((long long)p->B * p->heads > 65535) return fail(VEDA_ERR_INVALID_ARG, "B*heads exceeds 65535");
   return VEDA_OK;
 }
 
@@ -205,6 +206,18 @@ veda_status veda_tile_permute(const veda_problem* p, const void* x, void* xp, vo
   return ok();
 }
 
+veda_status veda_tile_permute_tripool(const veda_problem* p, const void* x, void* xp, float* desc, void* stream) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (!x || !xp || !desc) return fail(VEDA_ERR_INVALID_ARG, "x, xp and desc must be non-NULL");
+  if (!aligned16(x) || !aligned16(xp) || !aligned16(desc))
+    return fail(VEDA_ERR_INVALID_ARG, "x, xp and desc must be 16-byte aligned");
+  cudaError_t e = launch_permute_tripool(G, x, xp, desc, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "veda_tile_permute_tripool");
+  return ok();
+}
+
 veda_status veda_tile_unpermute(const veda_problem* p, const void* xp, void* x, void* stream) {
   Geometry G;
   veda_status s = make_geometry(p, &G);
@@ -231,7 +244,7 @@ veda_status veda_score_topk_workspace(const veda_problem* p, int32_t e, size_t* 
   Geometry G;
   veda_status s = make_geometry(p, &G);
   if (s != VEDA_OK) return s;
-  if (e < 4 || e > 128 || e % 4) return fail(VEDA_ERR_INVALID_ARG, "e must be a multiple of 4 in [4, 128] (got %d)", e);
+  if (e != 16 && e != 32 && e != 64 && e != 128) return fail(VEDA_ERR_INVALID_ARG, "e must be 16, 32, 64 or 128 (got %d)", e);
   if (!bytes) return fail(VEDA_ERR_INVALID_ARG, "bytes is NULL");
   *bytes = score_ws_bytes(G, e);
   return ok();
@@ -240,8 +253,10 @@ veda_status veda_score_topk_workspace(const veda_problem* p, int32_t e, size_t* 
 static veda_status check_mlp(const veda_mlp* m, const char* which) {
   if (!m) return fail(VEDA_ERR_INVALID_ARG, "%s estimator is NULL", which);
   if (!m->w1 || !m->b1 || !m->w2 || !m->b2) return fail(VEDA_ERR_INVALID_ARG, "%s estimator has a NULL weight", which);
-  if (m->hidden < 1 || m->hidden > 512) return fail(VEDA_ERR_INVALID_ARG, "hidden must be in [1, 512] (got %d)", m->hidden);
-  if (m->e < 4 || m->e > 128 || m->e % 4) return fail(VEDA_ERR_INVALID_ARG, "e must be a multiple of 4 in [4, 128] (got %d)", m->e);
+  if (m->hidden < 4 || m->hidden > 512 || m->hidden % 4)
+    return fail(VEDA_ERR_INVALID_ARG, "hidden must be a multiple of 4 in [4, 512] (got %d)", m->hidden);
+  if (m->e != 16 && m->e != 32 && m->e != 64 && m->e != 128)
+    return fail(VEDA_ERR_INVALID_ARG, "e must be 16, 32, 64 or 128 (got %d)", m->e);
   return VEDA_OK;
 }
 
@@ -270,7 +285,7 @@ veda_status veda_tile_score_topk(const veda_problem* p, const float* desc_q, con
   int qb, ntpad;
   size_t smem;
   score_topk_config(G.ntmax, e, &qb, &ntpad, &smem);
-  if (smem > 227 * 1024 || estimator_smem_bytes(G.d, hidden) > 227 * 1024)
+  if (smem > 227 * 1024 || estimator_smem_bytes(G.d, hidden, e) > 227 * 1024)
     return fail(VEDA_ERR_UNSUPPORTED, "NT_max = %d / hidden = %d exceed the shared-memory budget", G.ntmax, hidden);
   args.idx = idx;
   args.probs = probs;
@@ -297,6 +312,7 @@ veda_status veda_tile_sparse_attn(const veda_problem* p, const void* qp, const v
   if (!(std::isfinite(scale))) return fail(VEDA_ERR_INVALID_ARG, "scale must be finite");
   if (sparse_attn_smem_bytes(G.d, G.S, k_max) > 227 * 1024)
     return fail(VEDA_ERR_UNSUPPORTED, "k_max = %d exceeds the shared-memory budget", k_max);
+  if (G.ntmax > 32767) return fail(VEDA_ERR_UNSUPPORTED, "NT_max = %d exceeds 32767 tiles per head", G.ntmax);
   CUtensorMap tq, tk, tv;
   if ((s = encode_tile_major(G, qp, &tq)) != VEDA_OK || (s = encode_tile_major(G, kp, &tk)) != VEDA_OK ||
       (s = encode_tile_major(G, vp, &tv)) != VEDA_OK)

@@ -3,8 +3,9 @@
 ``VedaAttention`` owns the device buffers (torch allocations: memory
 plumbing only) and enqueues, on one CUDA stream,
 
-    veda_tile_permute(Q), (K), (V) -> veda_tripool(Qp), (Kp)
-    -> veda_tile_score_topk -> veda_tile_sparse_attn -> veda_tile_unpermute
+    veda_tile_permute_tripool(Q), (K)   (permute + TripPool in one pass)
+    -> veda_tile_permute(V) -> veda_tile_score_topk -> veda_tile_sparse_attn
+    -> veda_tile_unpermute
 
 which is the per-layer path of Veda's tile-sparse attention (technical
 summary, sections 2.1-2.3).  Every step runs in the library's kernels.
@@ -48,11 +49,9 @@ class VedaAttention:
     def select(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream=None) -> torch.Tensor:
         """Permute, pool and score; returns the selected tile indices."""
         p = self.p
-        B.veda_tile_permute(p, q, self.qp, stream)
-        B.veda_tile_permute(p, k, self.kp, stream)
+        B.veda_tile_permute_tripool(p, q, self.qp, self.desc_q, stream)
+        B.veda_tile_permute_tripool(p, k, self.kp, self.desc_k, stream)
         B.veda_tile_permute(p, v, self.vp, stream)
-        B.veda_tripool(p, self.qp, self.desc_q, stream)
-        B.veda_tripool(p, self.kp, self.desc_k, stream)
         B.veda_tile_score_topk(p, self.desc_q, self.desc_k, self.mlp_q, self.mlp_k, self.keep, self.idx, self.probs,
                                self.workspace, stream)
         return self.idx
