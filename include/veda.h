@@ -151,6 +151,26 @@ veda_status veda_tile_score_topk(const veda_problem* p, const float* desc_q, con
                                  int32_t* idx, int32_t k_max, float* probs, void* workspace,
                                  size_t workspace_bytes, void* stream);
 
+/* veda_tile_score_topk for callers that cannot provide device scratch memory
+ * -- a plugin whose host framework owns all device memory and gives it no
+ * workspace, or a latency-critical loop that must not call cudaMalloc (which
+ * can stall the whole device).  The paper has no counterpart; it is a
+ * deployment convenience.  Arguments, results and errors are those of
+ * veda_tile_score_topk, without the workspace: the estimator features live
+ * in a 16 MiB device array inside the library (2*B*heads*NT_max*e floats
+ * must fit; larger problems get VEDA_ERR_UNSUPPORTED and should use
+ * veda_tile_score_topk).  This call allocates nothing.  Every GPU that loads
+ * the library holds the array until the process exits.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) for that
+ * device; make that first call before any stream capture.  All calls share
+ * the one array, so calls that may overlap on the GPU (different streams,
+ * or different host threads on one device) race: serialise them.  Nothing
+ * needs clearing between calls -- every value read is written earlier in the
+ * same call. */
+veda_status veda_tile_score_topk_noalloc(const veda_problem* p, const float* desc_q, const float* desc_k,
+                                         const veda_mlp* mlp_q, const veda_mlp* mlp_k, float keep_ratio,
+                                         int32_t* idx, int32_t k_max, float* probs, void* stream);
+
 /* ---------------------------------------------------------------- step 5: tile-skipping attention */
 
 /* Block-sparse attention over only the selected K/V tiles (section 2.3,

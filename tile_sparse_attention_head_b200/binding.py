@@ -61,6 +61,8 @@ _SIG = {
     "veda_score_topk_workspace": [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)],
     "veda_tile_score_topk": [_P, _V, _V, ctypes.POINTER(veda_mlp), ctypes.POINTER(veda_mlp), ctypes.c_float, _V,
                              ctypes.c_int32, _V, _V, ctypes.c_size_t, _V],
+    "veda_tile_score_topk_noalloc": [_P, _V, _V, ctypes.POINTER(veda_mlp), ctypes.POINTER(veda_mlp), ctypes.c_float,
+                                     _V, ctypes.c_int32, _V, _V],
     "veda_tile_sparse_attn": [_P, _V, _V, _V, _V, ctypes.c_int32, ctypes.c_float, _V, _V, _V],
     "veda_tile_map_workspace": [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)],
     "veda_tile_map_maxpool": [_P, _V, _V, _V, ctypes.c_int32, ctypes.c_float, _V, _V, ctypes.c_size_t, _V],
@@ -215,6 +217,21 @@ def veda_tile_score_topk(p: Problem, desc_q: torch.Tensor, desc_k: torch.Tensor,
         _ptr(probs, "probs", torch.float32, (p.B, p.heads, p.nt_max, p.nt_max)),
         _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)),
         "veda_tile_score_topk")
+    return idx
+
+
+def veda_tile_score_topk_noalloc(p: Problem, desc_q: torch.Tensor, desc_k: torch.Tensor, mlp_q: veda_mlp,
+                                 mlp_k: veda_mlp, keep_ratio: float, idx: torch.Tensor,
+                                 probs: Optional[torch.Tensor], stream=None) -> torch.Tensor:
+    """veda_tile_score_topk without a workspace, for callers that cannot allocate device scratch."""
+    dshape = (p.B, p.heads, p.nt_max, 3 * p.d)
+    k_max = int(idx.shape[-1])
+    _check(LIB.veda_tile_score_topk_noalloc(
+        p.ref, _ptr(desc_q, "desc_q", torch.float32, dshape), _ptr(desc_k, "desc_k", torch.float32, dshape),
+        ctypes.byref(mlp_q), ctypes.byref(mlp_k), ctypes.c_float(keep_ratio),
+        _ptr(idx, "idx", torch.int32, (p.B, p.heads, p.nt_max, k_max)), k_max,
+        _ptr(probs, "probs", torch.float32, (p.B, p.heads, p.nt_max, p.nt_max)), _stream(stream)),
+        "veda_tile_score_topk_noalloc")
     return idx
 
 

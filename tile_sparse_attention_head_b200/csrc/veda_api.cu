@@ -298,6 +298,90 @@ veda_status veda_tile_score_topk(const veda_problem* p, const float* desc_q, con
   return ok();
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Scoring without a caller-provided workspace.
+//
+// Some callers cannot hand the library scratch memory: a plugin whose host
+// framework owns every byte of device memory and offers no workspace hook,
+// or a latency-critical loop that must not call cudaMalloc (it can stall the
+// whole device).  For them the estimator's per-tile features go to this
+// file-scope device array instead, sized for the largest workloads this
+// library is built for (16 MiB: the Wan2.1-14B 720p shape needs 14.1 MiB).
+// Every GPU that loads the library holds it until the process exits.
+// ---------------------------------------------------------------------------
+namespace veda {
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the host-side symbol is only a stand-in, never a device pointer).
+veda_status noalloc_scratch(float** out) {
+  constexpr int kMaxDevices = 64;
+  static float* ptrs[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "veda_tile_score_topk_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(VEDA_ERR_UNSUPPORTED, "device ordinal %d above %d", dev, kMaxDevices - 1);
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "veda_tile_score_topk_noalloc: cudaGetSymbolAddress");
+    ptrs[dev] = static_cast<float*>(p);
+  }
+  *out = ptrs[dev];
+  return VEDA_OK;
+}
+}  // namespace
+}  // namespace veda
+
+extern "C" {
+
+veda_status veda_tile_score_topk_noalloc(const veda_problem* p, const float* desc_q, const float* desc_k,
+                                         const veda_mlp* mlp_q, const veda_mlp* mlp_k, float keep_ratio,
+                                         int32_t* idx, int32_t k_max, float* probs, void* stream) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if ((s = check_mlp(mlp_q, "q")) != VEDA_OK || (s = check_mlp(mlp_k, "k")) != VEDA_OK) return s;
+  if (mlp_q->hidden != mlp_k->hidden || mlp_q->e != mlp_k->e)
+    return fail(VEDA_ERR_INVALID_ARG, "q and k estimators must have the same hidden and e");
+  if (!desc_q || !desc_k || !idx) return fail(VEDA_ERR_INVALID_ARG, "NULL tensor argument");
+  if (!aligned16(desc_q) || !aligned16(desc_k) || !aligned16(idx) || (probs && !aligned16(probs)))
+    return fail(VEDA_ERR_INVALID_ARG, "tensor arguments must be 16-byte aligned");
+  const int e = mlp_q->e, hidden = mlp_q->hidden;
+  const size_t need = score_ws_bytes(G, e);
+  if (need > kNoAllocScratchBytes)
+    return fail(VEDA_ERR_UNSUPPORTED,
+                "estimator scratch of %zu bytes exceeds the built-in %zu bytes (2*B*heads*NT_max*e floats); "
+                "use veda_tile_score_topk with a workspace",
+                need, kNoAllocScratchBytes);
+  TopkArgs args;
+  std::memset(&args, 0, sizeof(args));
+  int32_t kmax_needed = 0;
+  if ((s = keep_counts(G, keep_ratio, args.k_per_head, &kmax_needed)) != VEDA_OK) return s;
+  if (k_max < kmax_needed) return fail(VEDA_ERR_INVALID_ARG, "k_max = %d is below the largest keep count %d", k_max, kmax_needed);
+  int qb, ntpad;
+  size_t smem;
+  score_topk_config(G.ntmax, e, &qb, &ntpad, &smem);
+  if (smem > 227 * 1024 || estimator_smem_bytes(G.d, hidden, e) > 227 * 1024)
+    return fail(VEDA_ERR_UNSUPPORTED, "NT_max = %d / hidden = %d exceed the shared-memory budget", G.ntmax, hidden);
+  float* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != VEDA_OK) return s;
+  args.idx = idx;
+  args.probs = probs;
+  args.k_max = k_max;
+  EstimatorWeights wq{mlp_q->w1, mlp_q->b1, mlp_q->w2, mlp_q->b2};
+  EstimatorWeights wk{mlp_k->w1, mlp_k->b1, mlp_k->w2, mlp_k->b2};
+  cudaError_t ce = launch_score_topk(G, desc_q, desc_k, wq, wk, hidden, e, scratch, args, (cudaStream_t)stream);
+  if (ce != cudaSuccess) return cuda_fail(ce, "veda_tile_score_topk_noalloc");
+  return ok();
+}
+
 veda_status veda_tile_sparse_attn(const veda_problem* p, const void* qp, const void* kp, const void* vp,
                                   const int32_t* idx, int32_t k_max, float scale, void* op, float* lse,
                                   void* stream) {
