@@ -3,25 +3,34 @@
 // selected, non-contiguous K/V tiles and hides the data movement behind the
 // matrix math with warp-specialised producer/consumer roles).
 //
-// Blackwell design, one CTA per (b, h, Q tile), 6 warps:
-//   warp 0      TMA producer: the Q tile once, then K_j and V_j of every
-//               selected tile j into an NST-stage shared-memory ring (a
-//               permuted tile is S contiguous rows, so each fetch is a plain
-//               2D box; panels are 128-byte swizzled for the tensor cores);
-//   warp 1      tcgen05 issuer: S_t = Q K_t^T into one of three TMEM S/P
-//               buffers, then O += P_t V_t with P_t read straight from TMEM
-//               (the A operand of the "TS" form), O accumulating in TMEM;
-//               completions are signalled with tcgen05.commit on mbarriers.
-//               S_{t+1} is issued before P_t is ready so the tensor cores
-//               compute the next scores while the softmax runs;
-//   warps 2-5   softmax: one thread per query row loads its S row from TMEM,
-//               masks the pad keys of edge tiles, runs the online softmax in
-//               the log2 domain (a share of the exponentials on the FMA pipe),
-//               rescales its O row in TMEM only when the running maximum grows
-//               by more than 2^8, writes P as packed bf16 over its S row, and
-//               finally normalises O and stores it with the log-sum-exp.
-// TMEM: three S/P buffers (3 x 128 columns) + O (d columns) = 512 columns.
-// Shared memory: Q (S x d) + NST x (K + V) tiles; NST = 3 when it fits.
+// Blackwell design, one CTA per (b, h, Q tile), 12 warps in 3 warpgroups:
+//   warp 0       K producer: the Q tile once, then K_j of every selected tile
+//                j into a KST-stage shared-memory ring.  A permuted tile is S
+//                contiguous rows, so each fetch is a plain 2D TMA box; panels
+//                are 128-byte swizzled for the tensor cores.  A K stage is
+//                released as soon as the score product has read it.
+//   warp 2       V producer: V_j into a VST-stage ring, released after PV.
+//   warp 1       tcgen05 issuer of the score products S_t = Q K_t^T into the
+//                single TMEM S buffer, freed as soon as the owning stream has
+//                loaded S_t into registers.
+//   warp 3       tcgen05 issuer of the PV products O_s += P_t V_t (P read from
+//                TMEM, the "TS" form).  Each issuer's tcgen05.commit tracks
+//                only its own products.
+//   warps 4-7    softmax stream A: the tiles t = 0, 2, 4, ... of the list;
+//   warps 8-11   softmax stream B: the tiles t = 1, 3, 5, ...
+//                Each stream keeps its own online softmax (running maximum,
+//                row sum) and its own O accumulator, so the two warps that
+//                share a scheduler work on different tiles and never wait for
+//                each other; a thread owns one query row (its TMEM lane) and
+//                all BN columns of it.  Exponentials run in the log2 domain,
+//                a share of them on the FMA pipe; O is rescaled in TMEM only
+//                when the stream's maximum grows by more than 2^8; P is
+//                written as packed bf16 to the stream's own P buffer.
+//                At the end the two partial results are merged exactly:
+//                O = (2^(mA-m) O_A + 2^(mB-m) O_B) / (2^(mA-m) l_A + 2^(mB-m) l_B).
+// TMEM (512 columns): S (128), P_A and P_B (64 each), O_A and O_B (128 each).
+// Registers: the producer/issuer warpgroup gives registers back
+// (setmaxnreg) so the softmax warpgroups can hold a whole S row.
 // Every wait is bounded (veda_common.cuh); on a time-out every role leaves
 // its loop, in-flight copies and MMAs are drained and TMEM is freed.
 #include "veda_common.cuh"
@@ -34,35 +43,42 @@ namespace veda {
 constexpr int kPolyEvery = 4;
 constexpr int kSmemLimit = 232448;   // dynamic shared memory per CTA on sm_100
 
-template <int D, int BN, int NST>
+template <int D, int BN, int KST, int VST>
 struct AttnCfg {
   static constexpr int BM = 128;                 // MMA rows (query slots; S = 64 tiles use half)
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 384;
   static constexpr int kChunk = 128 * 128;       // one [128 rows x 128 B] swizzle panel
   static constexpr int kQBytes = BM * D * 2;
-  static constexpr int kKVBytes = BN * D * 2;
+  static constexpr int kTileBytes = BN * D * 2;  // one K or V tile
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + NST * kKVBytes;
-  static constexpr int kOffBar = kOffV + NST * kKVBytes;
-  static constexpr int kNumBars = 24;
-  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kOffV = kOffK + KST * kTileBytes;
+  static constexpr int kOffBar = kOffV + VST * kTileBytes;
+  static constexpr int kNumBars = 32;
+  static constexpr int kOffRed = kOffBar + kNumBars * 8;   // float [2 stream][2: m, l][128 rows]
+  static constexpr int kOffMisc = kOffRed + 2 * 2 * 128 * 4;
   static constexpr int kOffIdx = kOffMisc + 64;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kTmemO = 384;        // O accumulator column; S/P buffers at 0, 128, 256
+  static constexpr uint32_t kTmemS = 0;          // S, shared by the streams
+  static constexpr uint32_t kTmemP = 128;        // P of stream s at kTmemP + 64 s (packed bf16)
+  static constexpr uint32_t kTmemO = 256;        // O of stream s at kTmemO + 128 s
   static size_t smem_bytes(int k_max) { return 1024 + kOffIdx + 2 * (size_t)((k_max + 7) & ~7); }
 };
 
 // mbarrier slots
 enum {
   BAR_Q = 0,
-  BAR_KFULL = 1,    // +stage (<= 3)
-  BAR_VFULL = 4,    // +stage
-  BAR_KVEMPTY = 7,  // +stage
-  BAR_SFULL = 10,   // +S/P buffer (3)
-  BAR_PVDONE = 13,  // +S/P buffer (3): PV of the tile in that buffer completed
-  BAR_PFULL = 16,
-  BAR_DRAIN = 17
+  BAR_KFULL = 1,    // +stage (<= 4)
+  BAR_KEMPTY = 5,   // +stage
+  BAR_VFULL = 9,    // +stage (<= 4)
+  BAR_VEMPTY = 13,  // +stage
+  BAR_SFULL = 17,   // +stream: S of the stream's current tile is in TMEM
+  BAR_PFULL = 19,   // +stream: P of the stream's current tile is in TMEM (4 arrivals)
+  BAR_PVDONE = 21,  // +stream: the stream's last PV product completed
+  BAR_XFIN = 23,    // final (m, l) exchange between the streams
+  BAR_DRAIN = 24,   // score-product issuer drain
+  BAR_DRAIN2 = 25,  // PV-product issuer drain
+  BAR_SFREE = 26    // +stream: the stream has loaded its S from TMEM (4 arrivals)
 };
 
 // Warp-uniform bounded wait: every lane polls, the warp agrees on the result.
@@ -78,12 +94,34 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   mbar_wait(bar, parity, &dummy, timeout_ns);
 }
 
-template <int D, int BN, int NST>
-__global__ void __launch_bounds__(192, 1)
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* v) {
+  static_assert(N % 16 == 0, "");
+#pragma unroll
+  for (int c = 0; c + 32 <= N; c += 32) tmem_ld32(taddr + c, v + c);
+  if constexpr (N % 32 == 16) tmem_ld16(taddr + (N - 16), v + (N - 16));
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float* v) {
+#pragma unroll
+  for (int c = 0; c + 32 <= N; c += 32) tmem_st32(taddr + c, v + c);
+  if constexpr (N % 32 == 16) tmem_st16(taddr + (N - 16), v + (N - 16));
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_st_cols_u(uint32_t taddr, const uint32_t* v) {
+#pragma unroll
+  for (int c = 0; c + 32 <= N; c += 32) tmem_st32u(taddr + c, v + c);
+  if constexpr (N % 32 == 16) tmem_st16u(taddr + (N - 16), v + (N - 16));
+}
+
+template <int D, int BN, int KST, int VST>
+__global__ void __launch_bounds__(384, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Geometry G,
                        const __grid_constant__ AttnArgs A) {
-  using C = AttnCfg<D, BN, NST>;
+  using C = AttnCfg<D, BN, KST, VST>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -100,6 +138,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t sV = smem_u32(smem + C::kOffV);
   const uint32_t bar0 = smem_u32(smem + C::kOffBar);
   auto bar = [&](int b) { return bar0 + 8u * (uint32_t)b; };
+  float* red = reinterpret_cast<float*>(smem + C::kOffRed);
   int* misc = reinterpret_cast<int*>(smem + C::kOffMisc);  // [0] tmem base, [1] abort, [2] n_sel
   int16_t* s_idx = reinterpret_cast<int16_t*>(smem + C::kOffIdx);
   volatile int* abort = misc + 1;
@@ -117,28 +156,34 @@ __global__ void __launch_bounds__(192, 1)
   }
   if (tid == 0) {
     mbar_init(bar(BAR_Q), 1);
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < KST; ++s) {
       mbar_init(bar(BAR_KFULL + s), 1);
+      mbar_init(bar(BAR_KEMPTY + s), 1);
+    }
+    for (int s = 0; s < VST; ++s) {
       mbar_init(bar(BAR_VFULL + s), 1);
-      mbar_init(bar(BAR_KVEMPTY + s), 1);
+      mbar_init(bar(BAR_VEMPTY + s), 1);
     }
-    for (int b = 0; b < 3; ++b) {
-      mbar_init(bar(BAR_SFULL + b), 1);
-      mbar_init(bar(BAR_PVDONE + b), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(BAR_SFULL + s), 1);
+      mbar_init(bar(BAR_PFULL + s), 4);
+      mbar_init(bar(BAR_PVDONE + s), 1);
+      mbar_init(bar(BAR_SFREE + s), 4);
     }
-    mbar_init(bar(BAR_PFULL), 4);
+    mbar_init(bar(BAR_XFIN), 256);
     mbar_init(bar(BAR_DRAIN), 1);
+    mbar_init(bar(BAR_DRAIN2), 1);
     fence_mbar_init();
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&misc[0]), C::kTmemCols);
     tmem_relinquish();
   }
-  if (BN < 128 && warp >= 2) {
+  if (BN < 128 && warp >= 4) {
     // S = 64: the MMA always runs 128 rows; rows 64..127 of the Q panels are zero.
     for (int c = 0; c < D / 64; ++c) {
       uint4* p = reinterpret_cast<uint4*>(smem + C::kOffQ + c * C::kChunk + 64 * 128);
-      for (int e = tid - 64; e < 64 * 128 / 16; e += 128) p[e] = make_uint4(0, 0, 0, 0);
+      for (int e = tid - 128; e < 64 * 128 / 16; e += 256) p[e] = make_uint4(0, 0, 0, 0);
     }
     fence_proxy_async_smem();
   }
@@ -149,84 +194,89 @@ __global__ void __launch_bounds__(192, 1)
   const int n_sel = misc[2];
   const uint64_t tmo = A.timeout_ns;
 
+  if (warp < 4) {
+  // producers and issuers need few registers; the softmax warpgroups take them
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ K producer (+ Q)
     int issued = 0;
     bool q_issued = false;
     if (n_sel > 0) {
       if (lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
-        tma_prefetch_desc(&tmV);
         mbar_arrive_expect_tx(bar(BAR_Q), (uint32_t)(S * D * 2));
         for (int c = 0; c < D / 64; ++c)
           tma_load_2d(sQ + c * C::kChunk, &tmQ, bar(BAR_Q), 64 * c, (bh * G.ntmax + i) * S);
       }
       q_issued = true;
       for (int t = 0; t < n_sel; ++t) {
-        const int st = t % NST, fill = t / NST;
-        if (fill >= 1 && !warp_wait(bar(BAR_KVEMPTY + st), (fill - 1) & 1, abort, tmo)) break;
+        const int st = t % KST, fill = t / KST;
+        if (fill >= 1 && !warp_wait(bar(BAR_KEMPTY + st), (fill - 1) & 1, abort, tmo)) break;
         if (lane == 0) {
           const int y = (bh * G.ntmax + s_idx[t]) * S;
-          mbar_arrive_expect_tx(bar(BAR_KFULL + st), (uint32_t)C::kKVBytes);
+          mbar_arrive_expect_tx(bar(BAR_KFULL + st), (uint32_t)C::kTileBytes);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(sK + st * C::kKVBytes + c * BN * 128, &tmK, bar(BAR_KFULL + st), 64 * c, y);
-          mbar_arrive_expect_tx(bar(BAR_VFULL + st), (uint32_t)C::kKVBytes);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(sV + st * C::kKVBytes + c * BN * 128, &tmV, bar(BAR_VFULL + st), 64 * c, y);
+            tma_load_2d(sK + st * C::kTileBytes + c * BN * 128, &tmK, bar(BAR_KFULL + st), 64 * c, y);
         }
         __syncwarp();
         issued = t + 1;
       }
     }
     if (*abort) {
-      // Let every copy still in flight land before the CTA can exit.
       if (q_issued) drain_wait(bar(BAR_Q), 0, tmo);
-      for (int t = issued > NST ? issued - NST : 0; t < issued; ++t) {
-        drain_wait(bar(BAR_KFULL + t % NST), (t / NST) & 1, tmo);
-        drain_wait(bar(BAR_VFULL + t % NST), (t / NST) & 1, tmo);
-      }
+      for (int t = issued > KST ? issued - KST : 0; t < issued; ++t)
+        drain_wait(bar(BAR_KFULL + t % KST), (t / KST) & 1, tmo);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ tcgen05 issuer
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ V producer
+    int issued = 0;
     if (n_sel > 0) {
-      constexpr uint32_t idesc_qk = make_idesc_bf16(128, BN, false);
-      constexpr uint32_t idesc_pv = make_idesc_bf16(128, D, true);
-      auto issue_s = [&](int t) -> bool {
-        const int st = t % NST, b = t % 3;
-        if (!warp_wait(bar(BAR_KFULL + st), (t / NST) & 1, abort, tmo)) return false;
-        // The S/P buffer is free once the PV product of its previous tile is done.
-        if (t >= 3 && !warp_wait(bar(BAR_PVDONE + b), ((t / 3) - 1) & 1, abort, tmo)) return false;
-        tc_fence_after();
+      if (lane == 0) tma_prefetch_desc(&tmV);
+      for (int t = 0; t < n_sel; ++t) {
+        const int st = t % VST, fill = t / VST;
+        if (fill >= 1 && !warp_wait(bar(BAR_VEMPTY + st), (fill - 1) & 1, abort, tmo)) break;
         if (lane == 0) {
-          const uint32_t kbase = sK + st * C::kKVBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t da = make_sdesc_sw128(sQ + (kk >> 2) * C::kChunk + (kk & 3) * 32, 16, 1024);
-            const uint64_t db = make_sdesc_sw128(kbase + (kk >> 2) * BN * 128 + (kk & 3) * 32, 16, 1024);
-            umma_ss(tmem + b * 128, da, db, idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(bar(BAR_SFULL + b));
+          const int y = (bh * G.ntmax + s_idx[t]) * S;
+          mbar_arrive_expect_tx(bar(BAR_VFULL + st), (uint32_t)C::kTileBytes);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(sV + st * C::kTileBytes + c * BN * 128, &tmV, bar(BAR_VFULL + st), 64 * c, y);
         }
         __syncwarp();
-        return true;
-      };
-      bool ok = warp_wait(bar(BAR_Q), 0, abort, tmo) && issue_s(0);
+        issued = t + 1;
+      }
+    }
+    if (*abort) {
+      for (int t = issued > VST ? issued - VST : 0; t < issued; ++t)
+        drain_wait(bar(BAR_VFULL + t % VST), (t / VST) & 1, tmo);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ tcgen05 issuer, score products
+    if (n_sel > 0) {
+      constexpr uint32_t idesc_qk = make_idesc_bf16(128, BN, false);
+      // Descriptors are built once; per MMA only a compile-time offset (in
+      // 16-byte units, added to the start-address field) and the stage base
+      // change.
+      const uint64_t dq0 = make_sdesc_sw128(sQ, 16, 1024);
+      const uint64_t dk0 = make_sdesc_sw128(sK, 16, 1024);
+      bool ok = warp_wait(bar(BAR_Q), 0, abort, tmo);
       for (int t = 0; ok && t < n_sel; ++t) {
-        if (t + 1 < n_sel && !(ok = issue_s(t + 1))) break;
-        if (!(ok = warp_wait(bar(BAR_PFULL), t & 1, abort, tmo))) break;
-        if (!(ok = warp_wait(bar(BAR_VFULL + t % NST), (t / NST) & 1, abort, tmo))) break;
+        const int st = t % KST, s = t & 1;
+        if (!(ok = warp_wait(bar(BAR_KFULL + st), (t / KST) & 1, abort, tmo))) break;
+        // The single S buffer is free once the previous tile's stream has loaded it.
+        if (t >= 1 && !(ok = warp_wait(bar(BAR_SFREE + ((t - 1) & 1)), ((t - 1) >> 1) & 1, abort, tmo))) break;
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t vbase = sV + (t % NST) * C::kKVBytes;
-          const uint32_t pbase = tmem + (t % 3) * 128;
+          const uint64_t dk = dk0 + (uint64_t)((st * C::kTileBytes) >> 4);
+          const uint32_t dS = tmem + C::kTmemS;
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t db = make_sdesc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
-            umma_ts(tmem + C::kTmemO, pbase + kk * 8, db, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t da = dq0 + (uint64_t)(((kk >> 2) * C::kChunk + (kk & 3) * 32) >> 4);
+            const uint64_t db = dk + (uint64_t)(((kk >> 2) * BN * 128 + (kk & 3) * 32) >> 4);
+            umma_ss(dS, da, db, idesc_qk, kk > 0 ? 1u : 0u);
           }
-          umma_commit(bar(BAR_KVEMPTY + t % NST));
-          umma_commit(bar(BAR_PVDONE + t % 3));
+          umma_commit(bar(BAR_KEMPTY + st));
+          umma_commit(bar(BAR_SFULL + s));
         }
         __syncwarp();
       }
@@ -235,22 +285,61 @@ __global__ void __launch_bounds__(192, 1)
       __syncwarp();
       drain_wait(bar(BAR_DRAIN), 0, tmo);
     }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ tcgen05 issuer, PV products
+    if (n_sel > 0) {
+      constexpr uint32_t idesc_pv = make_idesc_bf16(128, D, true);
+      const uint64_t dv0 = make_sdesc_sw128(sV, BN * 128, 1024);
+      bool ok = true;
+      for (int t = 0; ok && t < n_sel; ++t) {
+        const int s = t & 1;
+        if (!(ok = warp_wait(bar(BAR_PFULL + s), (t >> 1) & 1, abort, tmo))) break;
+        if (!(ok = warp_wait(bar(BAR_VFULL + t % VST), (t / VST) & 1, abort, tmo))) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint64_t dv = dv0 + (uint64_t)(((t % VST) * C::kTileBytes) >> 4);
+          const uint32_t pbase = tmem + C::kTmemP + s * 64;
+          const uint32_t dO = tmem + C::kTmemO + s * 128;
+          const uint32_t acc0 = t >= 2 ? 1u : 0u;   // first tile of each stream starts its O
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint64_t db = dv + (uint64_t)((kk * 16 * 128) >> 4);
+            umma_ts(dO, pbase + kk * 8, db, idesc_pv, kk > 0 ? 1u : acc0);
+          }
+          umma_commit(bar(BAR_VEMPTY + t % VST));
+          umma_commit(bar(BAR_PVDONE + s));
+        }
+        __syncwarp();
+      }
+      if (lane == 0) umma_commit(bar(BAR_DRAIN2));
+      __syncwarp();
+      drain_wait(bar(BAR_DRAIN2), 0, tmo);
+    }
+  }
   } else {
-    // ------------------------------------------------------------ softmax warps
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;\n" ::: "memory");
+    // ------------------------------------------------------------ softmax streams
+    const int s = (warp - 4) >> 2;           // stream: tiles t with t % 2 == s
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t tS = t_lane + C::kTmemS;
+    const uint32_t tP = t_lane + C::kTmemP + s * 64;
+    const uint32_t tO = t_lane + C::kTmemO + s * 128;
     const float sl2 = A.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int t = 0; t < n_sel; ++t) {
-      const int b = t % 3;
-      if (!(ok = warp_wait(bar(BAR_SFULL + b), (t / 3) & 1, abort, tmo))) break;
+    for (int t = s; t < n_sel; t += 2) {
+      const int k = t >> 1;                  // this stream's k-th tile
+      if (!(ok = warp_wait(bar(BAR_SFULL + s), k & 1, abort, tmo))) break;
       tc_fence_after();
-      float s[BN];
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_lane + b * 128 + c * 32, &s[c * 32]);
+      float sc[BN];
+      tmem_ld_cols<BN>(tS, sc);
       tmem_ld_wait();
+      // S is in registers: the score issuer may overwrite the S buffer.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_SFREE + s));
 
       // Pad keys of an edge tile are masked out.
       const int j = s_idx[t];
@@ -268,24 +357,23 @@ __global__ void __launch_bounds__(192, 1)
         }
 #pragma unroll
         for (int c = 0; c < BN; ++c)
-          if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
+          if (!((mw[c >> 5] >> (c & 31)) & 1u)) sc[c] = -INFINITY;
       }
       // Row maximum over 8 independent chains.
       float m8[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) m8[q] = s[q];
+      for (int q = 0; q < 8; ++q) m8[q] = sc[q];
 #pragma unroll
       for (int c = 8; c < BN; c += 8)
 #pragma unroll
-        for (int q = 0; q < 8; ++q) m8[q] = fmaxf(m8[q], s[c + q]);
-      float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      mt *= sl2;
+        for (int q = 0; q < 8; ++q) m8[q] = fmaxf(m8[q], sc[c + q]);
+      const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
       // Lazy rescaling: keep the old reference maximum unless the new one is
       // more than 8 (log2 units) above it.
       float m_use;
       bool rescale = false;
-      if (t == 0) {
+      if (k == 0) {
         m_use = mt;
       } else if (mt > m_run + 8.0f) {
         m_use = mt;
@@ -300,8 +388,8 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t pk[BN / 2];
 #pragma unroll
       for (int c = 0; c < BN; c += 2) {
-        const float x0 = fmaf(s[c], sl2, -m_ref);
-        const float x1 = fmaf(s[c + 1], sl2, -m_ref);
+        const float x0 = fmaf(sc[c], sl2, -m_ref);
+        const float x1 = fmaf(sc[c + 1], sl2, -m_ref);
         const float p0 = (c % kPolyEvery == kPolyEvery - 1) ? exp2_fma(x0) : fast_exp2(x0);
         const float p1 = ((c + 1) % kPolyEvery == kPolyEvery - 1) ? exp2_fma(x1) : fast_exp2(x1);
         r8[c & 7] += p0;
@@ -313,62 +401,77 @@ __global__ void __launch_bounds__(192, 1)
       l_run = l_run * alpha + rs;
       m_run = m_use;
 
-      // P_t (bf16 pairs) over the S_t row in TMEM: the A operand of PV_t.
+      // The stream's previous PV must be done before its P buffer is
+      // rewritten and before its O is rescaled.
+      if (k >= 1 && !(ok = warp_wait(bar(BAR_PVDONE + s), (k - 1) & 1, abort, tmo))) break;
+      tc_fence_after();
+      // P (bf16 pairs) into the stream's P buffer: the A operand of PV.
+      tmem_st_cols_u<BN / 2>(tP, pk);
+      if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-      for (int c = 0; c < BN / 64; ++c) tmem_st32u(t_lane + b * 128 + c * 32, &pk[c * 32]);
-
-      // PV of the previous tile must be done before O is rescaled.
-      if (t >= 1) {
-        if (!(ok = warp_wait(bar(BAR_PVDONE + (t - 1) % 3), ((t - 1) / 3) & 1, abort, tmo))) break;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
+        for (int c = 0; c < D; c += 32) {
+          float o[32];
+          tmem_ld32(tO + c, o);
+          tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float o[32];
-            tmem_ld32(t_lane + C::kTmemO + c * 32, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int q = 0; q < 32; ++q) o[q] *= alpha;
-            tmem_st32(t_lane + C::kTmemO + c * 32, o);
-          }
+          for (int q = 0; q < 32; ++q) o[q] *= alpha;
+          tmem_st32(tO + c, o);
         }
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_PFULL));
+      if (lane == 0) mbar_arrive(bar(BAR_PFULL + s));
     }
-    // ------------------------------------------------------------ epilogue
-    if (ok && n_sel > 0) ok = warp_wait(bar(BAR_PVDONE + (n_sel - 1) % 3), ((n_sel - 1) / 3) & 1, abort, tmo);
+    // ------------------------------------------------------------ epilogue: merge the streams
+    const int n_s[2] = {(n_sel + 1) >> 1, n_sel >> 1};   // tiles per stream
+    // Own stream first: at most its last PV is pending (the one before it was
+    // observed in the loop), so the parity wait is exact.
+    if (ok && n_s[s] > 0) ok = warp_wait(bar(BAR_PVDONE + s), (n_s[s] - 1) & 1, abort, tmo);
+    if (ok) {
+      red[(s * 2 + 0) * 128 + row] = m_run;
+      red[(s * 2 + 1) * 128 + row] = l_run;
+      mbar_arrive(bar(BAR_XFIN));
+      ok = warp_wait(bar(BAR_XFIN), 0, abort, tmo);
+    }
+    // The other stream's warpgroup waited for its own last PV before the
+    // exchange, so that barrier is complete now and the wait returns at once.
+    if (ok && n_s[s ^ 1] > 0) ok = warp_wait(bar(BAR_PVDONE + (s ^ 1)), (n_s[s ^ 1] - 1) & 1, abort, tmo);
     if (ok) {
       tc_fence_after();
+      const float mA = red[0 * 128 + row], lA = red[1 * 128 + row];
+      const float mB = red[2 * 128 + row], lB = red[3 * 128 + row];
+      const float m = fmaxf(mA, mB);
+      const float wA = (lA > 0.f) ? fast_exp2(mA - m) : 0.f;
+      const float wB = (lB > 0.f) ? fast_exp2(mB - m) : 0.f;
+      const float l_tot = wA * lA + wB * lB;
+      const float inv_l = (l_tot > 0.f) ? 1.0f / l_tot : 0.f;
+      const float cA = wA * inv_l, cB = wB * inv_l;
+      // stream s writes output columns [s*D/2, (s+1)*D/2), reading both O's
       const long long grow = ((long long)bh * G.ntmax + i) * S + row;
-      const float inv_l = (l_run > 0.f) ? 1.0f / l_run : 0.f;
-      uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(A.op) + grow * D);
+      uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(A.op) + grow * D + s * (D / 2));
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float o[32];
-        if (n_sel > 0) {
-          tmem_ld32(t_lane + C::kTmemO + c * 32, o);
-          tmem_ld_wait();
-        } else {
+      for (int c = 0; c < D / 2; c += 32) {
+        float oa[32], ob[32];
+        tmem_ld32(t_lane + C::kTmemO + s * (D / 2) + c, oa);
+        tmem_ld32(t_lane + C::kTmemO + 128 + s * (D / 2) + c, ob);
+        tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 32; ++q) o[q] = 0.f;
-        }
+        for (int q = 0; q < 32; ++q) oa[q] = (cA != 0.f ? cA * oa[q] : 0.f) + (cB != 0.f ? cB * ob[q] : 0.f);
         if (row < S) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint4 v;
-            v.x = pack_bf16x2(o[q * 8 + 0] * inv_l, o[q * 8 + 1] * inv_l);
-            v.y = pack_bf16x2(o[q * 8 + 2] * inv_l, o[q * 8 + 3] * inv_l);
-            v.z = pack_bf16x2(o[q * 8 + 4] * inv_l, o[q * 8 + 5] * inv_l);
-            v.w = pack_bf16x2(o[q * 8 + 6] * inv_l, o[q * 8 + 7] * inv_l);
-            orow[c * 4 + q] = v;
+            v.x = pack_bf16x2(oa[q * 8 + 0], oa[q * 8 + 1]);
+            v.y = pack_bf16x2(oa[q * 8 + 2], oa[q * 8 + 3]);
+            v.z = pack_bf16x2(oa[q * 8 + 4], oa[q * 8 + 5]);
+            v.w = pack_bf16x2(oa[q * 8 + 6], oa[q * 8 + 7]);
+            orow[c / 8 + q] = v;
           }
         }
       }
-      if (A.lse != nullptr && row < S)
-        A.lse[grow] = (n_sel > 0) ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      if (A.lse != nullptr && s == 0 && row < S)
+        A.lse[grow] = (l_tot > 0.f) ? (m + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
     }
   }
 
@@ -380,32 +483,40 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-template <int D, int BN, int NST>
+template <int D, int BN, int KST, int VST>
 static cudaError_t launch_attn_t(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,
                                  const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s) {
-  using C = AttnCfg<D, BN, NST>;
+  using C = AttnCfg<D, BN, KST, VST>;
   const size_t smem = C::smem_bytes(a.k_max);
-  cudaError_t err = cudaFuncSetAttribute(sparse_attn_kernel<D, BN, NST>,
+  cudaError_t err = cudaFuncSetAttribute(sparse_attn_kernel<D, BN, KST, VST>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
+  // setmaxnreg moves registers between warpgroups inside the block's launch
+  // allocation: 128 threads drop to 56 and 256 threads rise to 224.  The
+  // split must fit the registers the block is launched with, or the raise
+  // would wait forever; refuse to launch otherwise.
+  cudaFuncAttributes attr;
+  if ((err = cudaFuncGetAttributes(&attr, sparse_attn_kernel<D, BN, KST, VST>)) != cudaSuccess) return err;
+  if (128 * 56 + 256 * 224 > C::kThreads * attr.numRegs) return cudaErrorInvalidConfiguration;
   const unsigned blocks = (unsigned)(G.B * G.heads * G.ntmax);
-  sparse_attn_kernel<D, BN, NST><<<blocks, C::kThreads, smem, s>>>(tq, tk, tv, G, a);
+  sparse_attn_kernel<D, BN, KST, VST><<<blocks, C::kThreads, smem, s>>>(tq, tk, tv, G, a);
   return cudaGetLastError();
 }
 
 template <int D, int BN>
 static cudaError_t launch_attn_d(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,
                                  const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s) {
-  if (AttnCfg<D, BN, 3>::smem_bytes(a.k_max) <= (size_t)kSmemLimit) return launch_attn_t<D, BN, 3>(G, tq, tk, tv, a, s);
-  return launch_attn_t<D, BN, 2>(G, tq, tk, tv, a, s);
+  if (AttnCfg<D, BN, 3, 2>::smem_bytes(a.k_max) <= (size_t)kSmemLimit)
+    return launch_attn_t<D, BN, 3, 2>(G, tq, tk, tv, a, s);
+  return launch_attn_t<D, BN, 2, 2>(G, tq, tk, tv, a, s);
 }
 
 size_t sparse_attn_smem_bytes(int d, int S, int k_max) {
-  // the smallest configuration that can run (two stages)
-  if (d == 128 && S == 128) return AttnCfg<128, 128, 2>::smem_bytes(k_max);
-  if (d == 128 && S == 64) return AttnCfg<128, 64, 2>::smem_bytes(k_max);
-  if (d == 64 && S == 128) return AttnCfg<64, 128, 2>::smem_bytes(k_max);
-  return AttnCfg<64, 64, 2>::smem_bytes(k_max);
+  // the smallest configuration that can run (two stages of each)
+  if (d == 128 && S == 128) return AttnCfg<128, 128, 2, 2>::smem_bytes(k_max);
+  if (d == 128 && S == 64) return AttnCfg<128, 64, 2, 2>::smem_bytes(k_max);
+  if (d == 64 && S == 128) return AttnCfg<64, 128, 2, 2>::smem_bytes(k_max);
+  return AttnCfg<64, 64, 2, 2>::smem_bytes(k_max);
 }
 
 cudaError_t launch_sparse_attn(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,

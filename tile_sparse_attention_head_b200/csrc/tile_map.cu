@@ -145,6 +145,9 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     constexpr uint32_t idesc = make_idesc_bf16(128, BN, false);
+    // Descriptors built once; per MMA only compile-time offsets are added.
+    const uint64_t dq0 = make_sdesc_sw128(sQ, 16, 1024);
+    const uint64_t dk0 = make_sdesc_sw128(sK, 16, 1024);
     bool ok = map_warp_wait(bar(MBAR_Q), 0, abort, tmo);
     for (int t = 0; ok && t < nt; ++t) {
       const int st = t % C::kStages, sb = t & 1;
@@ -152,12 +155,13 @@ __global__ void __launch_bounds__(192, 1)
       if (t >= 2 && !(ok = map_warp_wait(bar(MBAR_SFREE + sb), ((t >> 1) - 1) & 1, abort, tmo))) break;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t kbase = sK + st * C::kKBytes;
+        const uint64_t dk = dk0 + (uint64_t)((st * C::kKBytes) >> 4);
+        const uint32_t dS = tmem + sb * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t da = make_sdesc_sw128(sQ + (kk >> 2) * C::kChunk + (kk & 3) * 32, 16, 1024);
-          const uint64_t db = make_sdesc_sw128(kbase + (kk >> 2) * BN * 128 + (kk & 3) * 32, 16, 1024);
-          umma_ss(tmem + sb * 128, da, db, idesc, kk > 0 ? 1u : 0u);
+          const uint64_t da = dq0 + (uint64_t)(((kk >> 2) * C::kChunk + (kk & 3) * 32) >> 4);
+          const uint64_t db = dk + (uint64_t)(((kk >> 2) * BN * 128 + (kk & 3) * 32) >> 4);
+          umma_ss(dS, da, db, idesc, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(MBAR_KEMPTY + st));
         umma_commit(bar(MBAR_SFULL + sb));
