@@ -329,6 +329,16 @@ __global__ void __launch_bounds__(384, 1)
     const float sl2 = A.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
+    // Slot coordinates (t, y, x offsets) of this lane's key columns
+    // c = 32 w + lane, for the pad-key mask of edge tiles.
+    int8_t kt[BN / 32], ky[BN / 32], kx[BN / 32];
+#pragma unroll
+    for (int w = 0; w < BN / 32; ++w) {
+      const int c = w * 32 + lane;
+      kx[w] = (int8_t)(c % hg.pw);
+      ky[w] = (int8_t)((c / hg.pw) % hg.ph);
+      kt[w] = (int8_t)(c / (hg.pw * hg.ph));
+    }
     for (int t = s; t < n_sel; t += 2) {
       const int k = t >> 1;                  // this stream's k-th tile
       if (!(ok = warp_wait(bar(BAR_SFULL + s), k & 1, abort, tmo))) break;
@@ -350,25 +360,24 @@ __global__ void __launch_bounds__(384, 1)
       if (ct * ch * cw != S) {
         uint32_t mw[BN / 32];
 #pragma unroll
-        for (int w = 0; w < BN / 32; ++w) {
-          const int c = w * 32 + lane;
-          const int lw = c % hg.pw, lh = (c / hg.pw) % hg.ph, lt = c / (hg.pw * hg.ph);
-          mw[w] = __ballot_sync(0xffffffffu, lt < ct && lh < ch && lw < cw);
-        }
+        for (int w = 0; w < BN / 32; ++w) mw[w] = __ballot_sync(0xffffffffu, kt[w] < ct && ky[w] < ch && kx[w] < cw);
 #pragma unroll
         for (int c = 0; c < BN; ++c)
           if (!((mw[c >> 5] >> (c & 31)) & 1u)) sc[c] = -INFINITY;
       }
-      // Row maximum over 8 independent chains.
+      // Row maximum: three-input max over 8 independent chains.
       float m8[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) m8[q] = sc[q];
 #pragma unroll
-      for (int c = 8; c < BN; c += 8)
+      for (int c = 8; c + 16 <= BN; c += 16)
 #pragma unroll
-        for (int q = 0; q < 8; ++q) m8[q] = fmaxf(m8[q], sc[c + q]);
-      const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
+        for (int q = 0; q < 8; ++q) m8[q] = fmax3(m8[q], sc[c + q], sc[c + 8 + q]);
+      if constexpr (BN % 16 == 8) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) m8[q] = fmaxf(m8[q], sc[BN - 8 + q]);
+      }
+      const float mt = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * sl2;
       // Lazy rescaling: keep the old reference maximum unless the new one is
       // more than 8 (log2 units) above it.
       float m_use;
@@ -382,21 +391,28 @@ __global__ void __launch_bounds__(384, 1)
         m_use = m_run;
       }
       const float m_ref = (m_use == -INFINITY) ? 0.f : m_use;
-      float r8[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) r8[q] = 0.f;
+      // x = s*scale*log2(e) - m_ref as packed pairs; every kPolyEvery-th pair
+      // of exponentials on the FMA pipe; row sum over 4 packed chains.
+      const uint64_t scl2 = f2(sl2, sl2), nref2 = f2(-m_ref, -m_ref);
+      uint64_t r4[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[BN / 2];
 #pragma unroll
       for (int c = 0; c < BN; c += 2) {
-        const float x0 = fmaf(sc[c], sl2, -m_ref);
-        const float x1 = fmaf(sc[c + 1], sl2, -m_ref);
-        const float p0 = (c % kPolyEvery == kPolyEvery - 1) ? exp2_fma(x0) : fast_exp2(x0);
-        const float p1 = ((c + 1) % kPolyEvery == kPolyEvery - 1) ? exp2_fma(x1) : fast_exp2(x1);
-        r8[c & 7] += p0;
-        r8[(c + 1) & 7] += p1;
+        float x0, x1, p0, p1;
+        f2_split(f2_fma(f2(sc[c], sc[c + 1]), scl2, nref2), x0, x1);
+        if ((c >> 1) % kPolyEvery == kPolyEvery - 1) {
+          exp2_fma_x2(x0, x1, p0, p1);
+        } else {
+          p0 = fast_exp2(x0);
+          p1 = fast_exp2(x1);
+        }
+        r4[(c >> 1) & 3] = f2_add(r4[(c >> 1) & 3], f2(p0, p1));
         pk[c >> 1] = pack_bf16x2(p0, p1);
       }
-      const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+      float ra, rb, rc, rd;
+      f2_split(f2_add(r4[0], r4[1]), ra, rb);
+      f2_split(f2_add(r4[2], r4[3]), rc, rd);
+      const float rs = (ra + rb) + (rc + rd);
       const float alpha = rescale ? fast_exp2(m_run - m_ref) : 1.f;
       l_run = l_run * alpha + rs;
       m_run = m_use;

@@ -355,6 +355,53 @@ __device__ __forceinline__ float exp2_fma(float x) {
   return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
 }
 
+// Packed two-lane fp32 arithmetic (sm_100: fma/add.rn.f32x2 on a register pair).
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// exp2_fma on a pair of lanes: the reduction and the cubic run as packed
+// f32x2 operations, the exponent insertion per lane.
+__device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& y0, float& y1) {
+  x0 = fmaxf(x0, -126.0f);
+  x1 = fmaxf(x1, -126.0f);
+  const uint64_t x = f2(x0, x1);
+  const uint64_t magic = f2(12582912.0f, 12582912.0f);
+  const uint64_t nmagic = f2(-12582912.0f, -12582912.0f);
+  const uint64_t t = f2_add(x, magic);
+  float r0, r1, t0, t1;
+  f2_split(f2_add(t, nmagic), r0, r1);
+  const uint64_t f = f2_add(x, f2(-r0, -r1));
+  uint64_t p = f2_fma(f2(0.0551716685f, 0.0551716685f), f, f2(0.2426111251f, 0.2426111251f));
+  p = f2_fma(p, f, f2(0.6932609677f, 0.6932609677f));
+  p = f2_fma(p, f, f2(0.9999280572f, 0.9999280572f));
+  float p0, p1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  y0 = __int_as_float(__float_as_int(p0) + ((__float_as_int(t0) - 0x4B400000) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + ((__float_as_int(t1) - 0x4B400000) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
