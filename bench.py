@@ -1,10 +1,15 @@
 #!/usr/bin/env python3
 """Benchmark of the tile-sparse attention layer (Veda, head-aware tiles) on B200.
 
-One step = one attention layer of the inference path on one GPU:
+One step = one attention layer of the inference path on one GPU, all
+through the C ABI, inputs resident in HBM.  With ``--layout tile``:
     permute Q, K, V -> TripPool Q, K -> estimator + softmax + top-k
-    -> tile-skipping attention -> unpermute,
-all through the C ABI, inputs resident in HBM.  Default workload: the
+    -> tile-skipping attention -> unpermute;
+with ``--layout grid`` the permutation is folded into the attention kernel's
+tile fetch (each tile is one box of the grid-order tensor) and its output
+goes straight to grid rows:
+    TripPool Q, K (read in grid order) -> estimator + softmax + top-k
+    -> tile-skipping attention (grid order in and out).  Default workload: the
 Wan2.1-14B 720p/81-frame shape (21x45x80 grid = 75,600 tokens, 40 heads,
 d = 128, 128-token per-head tiles, keep 5% = 95% sparsity).
 
@@ -50,12 +55,12 @@ WORKLOAD_NAMES = {"wan14b": "Wan2.1-14B-720p-81f 21x45x80 (75,600 tokens) 40 hea
 # capture of the benchmarked launch (profiles/sparse_attn_wan14b.md), keyed by
 # workload and tied to the kernel source it was measured on: reported only
 # while csrc/sparse_attn.cu still hashes to that version.
-ATTN_TRAFFIC = {"wan14b": {"bytes": 1.26e9 + 858.49e6, "src_sha256_16": "b5a8f826b6c7f91f"}}
+ATTN_TRAFFIC = {("wan14b", "tile"): {"bytes": 1.26e9 + 858.49e6, "src_sha256_16": "b5a8f826b6c7f91f"}}
 
 
-def attn_traffic(workload: str):
+def attn_traffic(workload: str, layout: str):
     import hashlib
-    rec = ATTN_TRAFFIC.get(workload)
+    rec = ATTN_TRAFFIC.get((workload, layout))
     if rec is None:
         return None
     path = os.path.join(ROOT, "tile_sparse_attention_head_b200", "csrc", "sparse_attn.cu")
@@ -154,6 +159,17 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def bench_config(w, args, world, flops):
+    """The workload description shared by both arms' JSON lines."""
+    tensor_mb = w.B * w.heads * w.N * w.d * 2 / 1e6
+    return {"workload": WORKLOAD_NAMES.get(args.workload, args.workload), "preset": args.workload,
+            "grid": [w.T, w.H, w.W], "tokens": w.N, "heads": w.heads, "d": w.d, "S": w.S,
+            "keep": w.keep, "tilings": "per head from " + ",".join(str(t) for t in sorted(set(w.tilings))),
+            "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"replicas x{world}",
+            "kept_tile_flops_per_layer": flops, "layout": args.layout,
+            "l2": "inputs (3 x %.0f MB) larger than L2; no flush" % tensor_mb}
+
+
 def run_ours(args, world, rank, local):
     import tile_sparse_attention_head_b200 as V
     from veda_synth import PRESETS, make_mlp, make_qkv
@@ -164,31 +180,43 @@ def run_ours(args, world, rank, local):
     m = make_mlp(w, seed=1)
     dev = torch.device("cuda", torch.cuda.current_device())
     mlp = tuple(t.to(dev) for t in (m.w1, m.b1, m.w2, m.b2))
-    att = V.VedaAttention(p, mlp, mlp, w.keep, device=dev)
+    att = V.VedaAttention(p, mlp, mlp, w.keep, device=dev, layout=args.layout)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     out = torch.empty(p.grid_shape(), dtype=torch.bfloat16, device=dev)
     ks, _ = p.keep_count(w.keep)
     flops = kept_flops(p.nt_per_head, ks, w.B, w.S, w.d)
     stream = torch.cuda.current_stream()
 
-    # per-stage events for one instrumented step (after warm-up)
+    # The step's stages, in order, for per-stage events on one instrumented
+    # step (the same calls VedaAttention makes).
+    def score():
+        V.veda_tile_score_topk(p, att.desc_q, att.desc_k, att.mlp_q, att.mlp_k, att.keep, att.idx, None,
+                               att.workspace)
+
+    if args.layout == "tile":
+        stages = [("permute_tripool_qk", lambda: (V.veda_tile_permute_tripool(p, qd, att.qp, att.desc_q),
+                                                  V.veda_tile_permute_tripool(p, kd, att.kp, att.desc_k))),
+                  ("permute_v", lambda: V.veda_tile_permute(p, vd, att.vp)),
+                  ("score_topk", score),
+                  ("attention", lambda: V.veda_tile_sparse_attn(p, att.qp, att.kp, att.vp, att.idx, att.op)),
+                  ("unpermute", lambda: V.veda_tile_unpermute(p, att.op, out))]
+        launches_per_step = 7       # 2 permute+TripPool, permute, estimator, top-k, attention, unpermute
+    else:
+        stages = [("tripool_qk", lambda: (V.veda_tripool_grid(p, qd, att.desc_q),
+                                          V.veda_tripool_grid(p, kd, att.desc_k))),
+                  ("score_topk", score),
+                  ("attention", lambda: V.veda_tile_sparse_attn_grid(p, qd, kd, vd, att.idx, out))]
+        n_tilings = len(set(w.tilings))
+        launches_per_step = 4 + (n_tilings + 7) // 8   # 2 TripPool, estimator, top-k, attention per 8 tilings
+
     def step(ev=None):
         if ev is None:
             att(qd, kd, vd, out)
             return
         ev[0].record()
-        V.veda_tile_permute_tripool(p, qd, att.qp, att.desc_q)
-        V.veda_tile_permute_tripool(p, kd, att.kp, att.desc_k)
-        ev[1].record()
-        V.veda_tile_permute(p, vd, att.vp)
-        ev[2].record()
-        V.veda_tile_score_topk(p, att.desc_q, att.desc_k, att.mlp_q, att.mlp_k, att.keep, att.idx, None,
-                               att.workspace)
-        ev[3].record()
-        V.veda_tile_sparse_attn(p, att.qp, att.kp, att.vp, att.idx, att.op)
-        ev[4].record()
-        V.veda_tile_unpermute(p, att.op, out)
-        ev[5].record()
+        for si, (_, fn) in enumerate(stages):
+            fn()
+            ev[si + 1].record()
 
     for _ in range(args.warmup):
         step()
@@ -198,7 +226,7 @@ def run_ours(args, world, rank, local):
     clocks = Clocks(local)
     clocks.start()
     time.sleep(0.3)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
@@ -213,12 +241,8 @@ def run_ours(args, world, rank, local):
     V.veda_sync_status()
     ms_total = max_over_ranks(t0.elapsed_time(t1), world)
     ms_step = ms_total / args.steps
-    stage = {"permute_tripool_qk": [], "permute_v": [], "score_topk": [], "attention": [], "unpermute": []}
-    for ev in evs:
-        for name, a, b in (("permute_tripool_qk", 0, 1), ("permute_v", 1, 2), ("score_topk", 2, 3), ("attention", 3, 4),
-                           ("unpermute", 4, 5)):
-            stage[name].append(ev[a].elapsed_time(ev[b]))
-    stage_ms = {k: float(np.mean(v)) for k, v in stage.items()}
+    stage_ms = {name: float(np.mean([ev[si].elapsed_time(ev[si + 1]) for ev in evs]))
+                for si, (name, _) in enumerate(stages)}
     attn_ms = max_over_ranks(stage_ms["attention"], world)
 
     # ---- end to end through the public API with host buffers
@@ -252,22 +276,18 @@ def run_ours(args, world, rank, local):
     peaks, peak_src = load_peaks()
     achieved = flops / (attn_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "traffic": attn_traffic(args.workload),
+                "frac": achieved / peaks["bf16_tflops"], "traffic": attn_traffic(args.workload, args.layout),
                 "traffic_unit": "bytes per launch (DRAM read + write)",
-                "kernel": "sparse_attn_kernel<128,128,3,2>", "peak_source": f"{peak_src} bf16 burst",
+                "kernel": f"sparse_attn_kernel<{w.d},{w.S},3,2,{'grid' if args.layout == 'grid' else 'tile'}>",
+                "peak_source": f"{peak_src} bf16 burst",
                 "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]}
     res = {"metric": METRIC, "value": world * flops / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-           "config": {"workload": WORKLOAD_NAMES.get(args.workload, args.workload), "preset": args.workload,
-                      "grid": [w.T, w.H, w.W], "tokens": w.N, "heads": w.heads, "d": w.d, "S": w.S,
-                      "keep": w.keep, "tilings": "per head from {(2,8,8),(1,8,16),(8,4,4),(4,4,8)}",
-                      "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"replicas x{world}",
-                      "kept_tile_flops_per_layer": flops,
-                      "l2": "inputs (3 x %.0f MB) larger than L2; no flush" % (q.numel() * 2 / 1e6)},
+           "config": bench_config(w, args, world, flops),
            "ms_per_layer": ms_step, "stage_ms": stage_ms, "attn_tflops": achieved,
            "pct_of_bf16_peak": 100.0 * achieved / peaks["bf16_tflops"],
-           "roofline": roofline, "gpu_launches": 7 * args.steps, "clocks": clk, "e2e": e2e}
+           "roofline": roofline, "gpu_launches": launches_per_step * args.steps, "clocks": clk, "e2e": e2e}
     return res, (w, p, ks, flops)
 
 
@@ -319,11 +339,11 @@ def run_reference(args, world, rank):
         flops += f
     value = flops / secs / 1e12
     cores = os.cpu_count()
+    layer_flops = kept_flops(nts, ks, w.B, w.S, w.d)
     return {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": WORKLOAD_NAMES.get(args.workload, args.workload), "preset": args.workload,
-                       "parallelism": "cpu"},
+            "config": bench_config(w, args, world, layer_flops),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -335,6 +355,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="wan14b")
+    ap.add_argument("--layout", choices=["tile", "grid"], default="grid",
+                    help="tile-major copies (permute/unpermute steps) or grid order throughout")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tiles", type=int, default=24, help="Q tiles per oracle sample (reference arm)")

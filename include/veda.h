@@ -8,6 +8,11 @@
  *   veda_tile_permute (Q, K, V)  ->  veda_tripool (Q, K)  ->  veda_tile_score_topk
  *   ->  veda_tile_sparse_attn  ->  veda_tile_unpermute
  *
+ * or, with the permutation folded into the attention kernel's tile fetch and
+ * no tile-major copies at all,
+ *
+ *   veda_tripool_grid (Q, K)  ->  veda_tile_score_topk  ->  veda_tile_sparse_attn_grid
+ *
  * and the distillation target is built by veda_tile_map_maxpool.
  *
  * Conventions shared by every call
@@ -127,6 +132,12 @@ veda_status veda_tripool(const veda_problem* p, const void* xp, float* desc, voi
 veda_status veda_tile_permute_tripool(const veda_problem* p, const void* x, void* xp, float* desc,
                                       void* stream);
 
+/* TripPool straight from a grid-order tensor: x [B, heads, N, d] bf16 (read),
+ * desc [B, heads, NT_max, 3d] fp32 (written in full), equal to veda_tripool
+ * of veda_tile_permute(x); no permuted copy is made.  x and desc must not
+ * overlap. */
+veda_status veda_tripool_grid(const veda_problem* p, const void* x, float* desc, void* stream);
+
 /* ---------------------------------------------------------------- steps 3-4: estimator + top-k */
 
 /* Bytes of workspace veda_tile_score_topk needs for estimator width e. */
@@ -189,6 +200,19 @@ veda_status veda_tile_score_topk_noalloc(const veda_problem* p, const float* des
 veda_status veda_tile_sparse_attn(const veda_problem* p, const void* qp, const void* kp,
                                   const void* vp, const int32_t* idx, int32_t k_max, float scale,
                                   void* op, float* lse, void* stream);
+
+/* The same attention on grid-order tensors (section 2.2's head-aware tiling
+ * applied inside the kernel; the output goes straight back to grid order).
+ * q, k, v [B, heads, N, d] bf16 (read); idx, k_max and scale as in
+ * veda_tile_sparse_attn.  Each selected tile is fetched as one pt x ph x pw
+ * box of the grid, so the result equals veda_tile_unpermute of
+ * veda_tile_sparse_attn on the permuted tensors: o [B, heads, N, d] bf16,
+ * every row written; lse [B, heads, N] fp32 or NULL, every entry written.
+ * o must not overlap q, k or v.  Heads are grouped by tiling; one launch
+ * covers up to 8 distinct tilings, so more tilings take several launches. */
+veda_status veda_tile_sparse_attn_grid(const veda_problem* p, const void* q, const void* k,
+                                       const void* v, const int32_t* idx, int32_t k_max, float scale,
+                                       void* o, float* lse, void* stream);
 
 /* ---------------------------------------------------------------- secondary: tile map */
 

@@ -22,6 +22,7 @@ import numpy as np
 import torch
 
 from oracle import veda_oracle as O
+from veda_synth import PRESETS, Workload
 
 ATTN_MAX_ABS = 1e-2
 ATTN_REL_L2 = 5e-3
@@ -31,6 +32,28 @@ PROBS_REL = 2e-4
 PROBS_ABS = 1e-7
 MAP_REL = 1e-3
 NEAR_TIE = 1e-4
+
+
+def wl(name, grid, B, heads, d, S, tilings, keep, hidden, e, bias=None) -> Workload:
+    return Workload(name=name, T=grid[0], H=grid[1], W=grid[2], B=B, heads=heads, d=d, S=S,
+                    tilings=tuple(tilings), keep=keep, hidden=hidden, e=e, bias=bias)
+
+
+# Small problems the oracle finishes in seconds: several tiles per axis,
+# ragged tiles on every face, both tile sizes and head dims, B = 2.
+SMALL = [
+    PRESETS["tiny"],
+    wl("odd64", (5, 13, 19), 1, 3, 64, 64, [(1, 8, 8), (4, 4, 4), (2, 4, 8)], 0.25, 128, 32, "rff"),
+    wl("odd128", (5, 19, 27), 2, 4, 128, 128, [(2, 8, 8), (1, 8, 16), (8, 4, 4), (4, 4, 8)], 0.2, 256, 64, "rff"),
+    wl("d64s128", (6, 12, 20), 1, 2, 64, 128, [(2, 8, 8), (4, 4, 8)], 0.3, 128, 32),
+    wl("d128s64", (4, 16, 16), 1, 2, 128, 64, [(1, 8, 8), (4, 4, 4)], 0.5, 256, 64, "local"),
+]
+
+# Ten distinct tilings of S = 64 (more than one grid-order attention launch
+# covers), several with a factor larger than the grid dimension it tiles.
+MANY_TILINGS = wl("many64", (5, 13, 19), 1, 10, 64, 64,
+                  [(1, 8, 8), (4, 4, 4), (2, 4, 8), (8, 8, 1), (8, 1, 8), (1, 4, 16), (16, 2, 2), (2, 8, 4),
+                   (4, 2, 8), (1, 2, 32)], 0.25, 128, 32, "rff")
 
 
 def f64(t: torch.Tensor) -> np.ndarray:

@@ -87,7 +87,13 @@ def test_invalid_arguments_are_rejected_on_the_host(V):
     assert lib.veda_tile_permute(p.ref, None, None, None) == B.VEDA_ERR_INVALID_ARG
     assert lib.veda_tripool(p.ref, None, None, None) == B.VEDA_ERR_INVALID_ARG
     assert lib.veda_tile_sparse_attn(p.ref, None, None, None, None, 1, 0.0, None, None, None) == B.VEDA_ERR_INVALID_ARG
+    assert lib.veda_tripool_grid(p.ref, None, None, None) == B.VEDA_ERR_INVALID_ARG
+    assert (lib.veda_tile_sparse_attn_grid(p.ref, None, None, None, None, 1, 0.0, None, None, None)
+            == B.VEDA_ERR_INVALID_ARG)
     assert b"non-NULL" in lib.veda_last_error() or b"NULL" in lib.veda_last_error()
+    # k_max < 1 and misaligned grid-order pointers (never dereferenced on the host)
+    assert lib.veda_tile_sparse_attn_grid(p.ref, 256, 256, 256, 256, 0, 0.0, 256, None, None) == B.VEDA_ERR_INVALID_ARG
+    assert lib.veda_tile_sparse_attn_grid(p.ref, 8, 256, 256, 256, 1, 0.0, 256, None, None) == B.VEDA_ERR_INVALID_ARG
     # misaligned pointers are refused too
     assert lib.veda_tile_permute(p.ref, 8, 16, None) == B.VEDA_ERR_INVALID_ARG
     assert lib.veda_set_wait_timeout_ns(0) == B.VEDA_ERR_INVALID_ARG

@@ -58,12 +58,14 @@ _SIG = {
     "veda_tile_unpermute": [_P, _V, _V, _V],
     "veda_tile_permute_tripool": [_P, _V, _V, _V, _V],
     "veda_tripool": [_P, _V, _V, _V],
+    "veda_tripool_grid": [_P, _V, _V, _V],
     "veda_score_topk_workspace": [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)],
     "veda_tile_score_topk": [_P, _V, _V, ctypes.POINTER(veda_mlp), ctypes.POINTER(veda_mlp), ctypes.c_float, _V,
                              ctypes.c_int32, _V, _V, ctypes.c_size_t, _V],
     "veda_tile_score_topk_noalloc": [_P, _V, _V, ctypes.POINTER(veda_mlp), ctypes.POINTER(veda_mlp), ctypes.c_float,
                                      _V, ctypes.c_int32, _V, _V],
     "veda_tile_sparse_attn": [_P, _V, _V, _V, _V, ctypes.c_int32, ctypes.c_float, _V, _V, _V],
+    "veda_tile_sparse_attn_grid": [_P, _V, _V, _V, _V, ctypes.c_int32, ctypes.c_float, _V, _V, _V],
     "veda_tile_map_workspace": [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)],
     "veda_tile_map_maxpool": [_P, _V, _V, _V, ctypes.c_int32, ctypes.c_float, _V, _V, ctypes.c_size_t, _V],
     "veda_sync_status": [_V],
@@ -188,6 +190,14 @@ def veda_tripool(p: Problem, xp: torch.Tensor, desc: torch.Tensor, stream=None) 
     return desc
 
 
+def veda_tripool_grid(p: Problem, x: torch.Tensor, desc: torch.Tensor, stream=None) -> torch.Tensor:
+    _check(LIB.veda_tripool_grid(p.ref, _ptr(x, "x", torch.bfloat16, p.grid_shape()),
+                                 _ptr(desc, "desc", torch.float32, (p.B, p.heads, p.nt_max, 3 * p.d)),
+                                 _stream(stream)),
+           "veda_tripool_grid")
+    return desc
+
+
 def veda_score_topk_workspace(p: Problem, e: int) -> int:
     n = ctypes.c_size_t()
     _check(LIB.veda_score_topk_workspace(p.ref, int(e), ctypes.byref(n)), "veda_score_topk_workspace")
@@ -247,6 +257,20 @@ def veda_tile_sparse_attn(p: Problem, qp: torch.Tensor, kp: torch.Tensor, vp: to
         _ptr(lse, "lse", torch.float32, (p.B, p.heads, p.nt_max * p.S)), _stream(stream)),
         "veda_tile_sparse_attn")
     return op
+
+
+def veda_tile_sparse_attn_grid(p: Problem, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor,
+                               o: torch.Tensor, lse: Optional[torch.Tensor] = None, scale: float = 0.0,
+                               stream=None) -> torch.Tensor:
+    gs = p.grid_shape()
+    k_max = int(idx.shape[-1])
+    _check(LIB.veda_tile_sparse_attn_grid(
+        p.ref, _ptr(q, "q", torch.bfloat16, gs), _ptr(k, "k", torch.bfloat16, gs),
+        _ptr(v, "v", torch.bfloat16, gs), _ptr(idx, "idx", torch.int32, (p.B, p.heads, p.nt_max, k_max)), k_max,
+        ctypes.c_float(scale), _ptr(o, "o", torch.bfloat16, gs),
+        _ptr(lse, "lse", torch.float32, (p.B, p.heads, p.N)), _stream(stream)),
+        "veda_tile_sparse_attn_grid")
+    return o
 
 
 def veda_tile_map_workspace(p: Problem, R: int) -> int:

@@ -28,9 +28,23 @@ struct AttnArgs {
   const int32_t* idx;
   int32_t k_max;
   float scale_log2;   // softmax scale * log2(e)
-  void* op;           // bf16 [B, heads, NT_max*S, d]
-  float* lse;         // fp32 [B, heads, NT_max*S] or null
+  void* op;           // bf16 [B, heads, NT_max*S, d] (tile-major) or [B, heads, N, d] (grid order)
+  float* lse;         // fp32 [B, heads, NT_max*S] or [B, heads, N]; or null
   uint64_t timeout_ns;
+  // Grid-order launches only: the heads this launch covers and, per head,
+  // which of the launch's tensor maps holds its tile box.
+  int32_t n_group;
+  int16_t head_list[VEDA_MAX_HEADS];
+  int8_t map_of_head[VEDA_MAX_HEADS];
+};
+
+// Tensor maps of one attention launch.  Tile-major operands need one map
+// each; grid-order operands need one per distinct tiling (the tile box is
+// part of the map), up to kMaxGridMaps per launch.
+constexpr int kMaxGridMaps = 8;
+template <int NM>
+struct AttnMaps {
+  CUtensorMap q[NM], k[NM], v[NM];
 };
 
 struct MapArgs {
@@ -58,6 +72,12 @@ cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const floa
 
 cudaError_t launch_sparse_attn(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
+// Grid-order variant: Q/K/V tiles are fetched as 5D boxes of the grid-order
+// tensors, O and the LSE are written to grid rows.  One launch covers the
+// heads a.head_list[0..a.n_group); head h uses maps m.*[a.map_of_head[h]].
+cudaError_t launch_sparse_attn_grid(const Geometry& G, const AttnMaps<kMaxGridMaps>& m, const AttnArgs& a,
+                                    cudaStream_t s);
+cudaError_t launch_tripool_grid(const Geometry& G, const void* x, float* desc, cudaStream_t s);
 
 cudaError_t launch_tile_map(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,
                             const MapArgs& a, cudaStream_t s);

@@ -74,9 +74,11 @@ __device__ __forceinline__ void tripool_reduce_store(const Stats8& st, float* re
   }
 }
 
-// grid: (NT_max, B*heads).  Writes all S rows of tile j of head h (zeros for
-// pad slots and tiles j >= NT_h); with POOL also desc[b, h, j, :].
-template <int D, int S, bool POOL>
+// grid: (NT_max, B*heads).  Gathers tile j of head h from the grid-order
+// tensor.  With WRITE, writes all S rows of it (zeros for pad slots and tiles
+// j >= NT_h); with POOL, also desc[b, h, j, :].  POOL without WRITE is the
+// TripPool of a grid-order tensor (no permuted copy is made).
+template <int D, int S, bool POOL, bool WRITE = true>
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(const __grid_constant__ Geometry G,
                                                                const uint4* __restrict__ x,
                                                                uint4* __restrict__ xp,
@@ -96,7 +98,6 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const __grid_cons
   __syncthreads();
 
   const uint4* xb = x + (size_t)bh * G.N * CPR;
-  uint4* xo = xp + ((size_t)bh * G.ntmax + j) * (size_t)S * CPR;
   const int chunk = tid % CPR, r0 = tid / CPR;
   uint4 v[PASSES];
 #pragma unroll
@@ -104,8 +105,11 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const __grid_cons
     const int n = s_src[r0 + p * RPP];
     v[p] = (n >= 0) ? __ldg(xb + (size_t)n * CPR + chunk) : make_uint4(0u, 0u, 0u, 0u);
   }
+  if constexpr (WRITE) {
+    uint4* xo = xp + ((size_t)bh * G.ntmax + j) * (size_t)S * CPR;
 #pragma unroll
-  for (int p = 0; p < PASSES; ++p) xo[(size_t)(r0 + p * RPP) * CPR + chunk] = v[p];
+    for (int p = 0; p < PASSES; ++p) xo[(size_t)(r0 + p * RPP) * CPR + chunk] = v[p];
+  }
 
   if constexpr (POOL) {
     float* out = desc + ((size_t)bh * G.ntmax + j) * 3 * D;
@@ -213,6 +217,16 @@ cudaError_t launch_unpermute(const Geometry& G, const void* xp, void* x, cudaStr
   dim3 grid((G.N + 127) / 128, G.B * G.heads);
   if (G.d == 128) unpermute_kernel<128><<<grid, kPermThreads, 0, s>>>(G, (const uint4*)xp, (uint4*)x);
   else unpermute_kernel<64><<<grid, kPermThreads, 0, s>>>(G, (const uint4*)xp, (uint4*)x);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tripool_grid(const Geometry& G, const void* x, float* desc, cudaStream_t s) {
+  dim3 grid(G.ntmax, G.B * G.heads);
+  const uint4* xi = (const uint4*)x;
+  if (G.d == 128 && G.S == 128) permute_kernel<128, 128, true, false><<<grid, kPermThreads, 0, s>>>(G, xi, nullptr, desc);
+  else if (G.d == 128) permute_kernel<128, 64, true, false><<<grid, kPermThreads, 0, s>>>(G, xi, nullptr, desc);
+  else if (G.S == 128) permute_kernel<64, 128, true, false><<<grid, kPermThreads, 0, s>>>(G, xi, nullptr, desc);
+  else permute_kernel<64, 64, true, false><<<grid, kPermThreads, 0, s>>>(G, xi, nullptr, desc);
   return cudaGetLastError();
 }
 

@@ -6,9 +6,11 @@
 // Blackwell design, one CTA per (b, h, Q tile), 12 warps in 3 warpgroups:
 //   warp 0       K producer: the Q tile once, then K_j of every selected tile
 //                j into a KST-stage shared-memory ring.  A permuted tile is S
-//                contiguous rows, so each fetch is a plain 2D TMA box; panels
-//                are 128-byte swizzled for the tensor cores.  A K stage is
-//                released as soon as the score product has read it.
+//                contiguous rows, so each fetch is a plain 2D TMA box; on
+//                grid-order tensors it is one 5D box (the tile's pt x ph x pw
+//                tokens), which lands in shared memory in the same slot order.
+//                Panels are 128-byte swizzled for the tensor cores.  A K stage
+//                is released as soon as the score product has read it.
 //   warp 2       V producer: V_j into a VST-stage ring, released after PV.
 //   warp 1       tcgen05 issuer of the score products S_t = Q K_t^T into the
 //                single TMEM S buffer, freed as soon as the owning stream has
@@ -116,22 +118,50 @@ __device__ __forceinline__ void tmem_st_cols_u(uint32_t taddr, const uint32_t* v
   if constexpr (N % 32 == 16) tmem_st16u(taddr + (N - 16), v + (N - 16));
 }
 
-template <int D, int BN, int KST, int VST>
+// GRID = false: Q/K/V/O are tile-major [B, heads, NT_max*S, d]; tile j of a
+// head is rows j*S .. j*S+S-1, fetched as one 2D box per 64 channels.
+// GRID = true: Q/K/V/O stay in grid order [B, heads, T*H*W, d].  Seen as the
+// 5D array [B*heads, T, H, W, d], tile j of a head with tiling (pt, ph, pw)
+// is the box of pt x ph x pw tokens at (jt*pt, jh*ph, jw*pw); TMA writes the
+// box to shared memory with w fastest, then h, then t -- exactly the
+// within-tile slot order -- and fills the part of an edge box that lies
+// outside the grid with zeros, as the permutation does for pad slots.  O and
+// the LSE of each valid query slot are written straight to its grid row.
+template <int D, int BN, int KST, int VST, bool GRID>
 __global__ void __launch_bounds__(384, 1)
-    sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Geometry G,
-                       const __grid_constant__ AttnArgs A) {
+    sparse_attn_kernel(const __grid_constant__ AttnMaps<GRID ? kMaxGridMaps : 1> M,
+                       const __grid_constant__ Geometry G, const __grid_constant__ AttnArgs A) {
   using C = AttnCfg<D, BN, KST, VST>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int i = blockIdx.x % G.ntmax;
-  const int bh = blockIdx.x / G.ntmax;
-  const int h = bh % G.heads;
+  int h, bh, mi = 0;
+  if constexpr (GRID) {
+    const int hb = blockIdx.x / G.ntmax;        // b * n_group + position in the head list
+    h = A.head_list[hb % A.n_group];
+    bh = (hb / A.n_group) * G.heads + h;
+    mi = A.map_of_head[h];
+  } else {
+    bh = blockIdx.x / G.ntmax;
+    h = bh % G.heads;
+  }
   const HeadGeom hg = G.g[h];
   if (i >= hg.nt) return;  // CTA-uniform, before any barrier or TMEM use
   const int S = G.S;
+  const CUtensorMap* tmQ = &M.q[mi];
+  const CUtensorMap* tmK = &M.k[mi];
+  const CUtensorMap* tmV = &M.v[mi];
+  // Channel chunk c (64 channels) of tile j into shared memory at dst.
+  auto load_tile = [&](uint32_t dst, const CUtensorMap* map, uint32_t b, int c, int j) {
+    if constexpr (GRID) {
+      const int jw = j % hg.nTw, jh = (j / hg.nTw) % hg.nTh, jt = j / (hg.nTw * hg.nTh);
+      tma_load_5d(dst, map, b, 64 * c, jw * hg.pw, jh * hg.ph, jt * hg.pt, bh);
+    } else {
+      tma_load_2d(dst, map, b, 64 * c, (bh * G.ntmax + j) * S);
+    }
+  };
 
   const uint32_t sQ = smem_u32(smem + C::kOffQ);
   const uint32_t sK = smem_u32(smem + C::kOffK);
@@ -203,21 +233,20 @@ __global__ void __launch_bounds__(384, 1)
     bool q_issued = false;
     if (n_sel > 0) {
       if (lane == 0) {
-        tma_prefetch_desc(&tmQ);
-        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(tmQ);
+        tma_prefetch_desc(tmK);
         mbar_arrive_expect_tx(bar(BAR_Q), (uint32_t)(S * D * 2));
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_2d(sQ + c * C::kChunk, &tmQ, bar(BAR_Q), 64 * c, (bh * G.ntmax + i) * S);
+        for (int c = 0; c < D / 64; ++c) load_tile(sQ + c * C::kChunk, tmQ, bar(BAR_Q), c, i);
       }
       q_issued = true;
       for (int t = 0; t < n_sel; ++t) {
         const int st = t % KST, fill = t / KST;
         if (fill >= 1 && !warp_wait(bar(BAR_KEMPTY + st), (fill - 1) & 1, abort, tmo)) break;
         if (lane == 0) {
-          const int y = (bh * G.ntmax + s_idx[t]) * S;
+          const int j = s_idx[t];
           mbar_arrive_expect_tx(bar(BAR_KFULL + st), (uint32_t)C::kTileBytes);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(sK + st * C::kTileBytes + c * BN * 128, &tmK, bar(BAR_KFULL + st), 64 * c, y);
+            load_tile(sK + st * C::kTileBytes + c * BN * 128, tmK, bar(BAR_KFULL + st), c, j);
         }
         __syncwarp();
         issued = t + 1;
@@ -232,15 +261,15 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------------------ V producer
     int issued = 0;
     if (n_sel > 0) {
-      if (lane == 0) tma_prefetch_desc(&tmV);
+      if (lane == 0) tma_prefetch_desc(tmV);
       for (int t = 0; t < n_sel; ++t) {
         const int st = t % VST, fill = t / VST;
         if (fill >= 1 && !warp_wait(bar(BAR_VEMPTY + st), (fill - 1) & 1, abort, tmo)) break;
         if (lane == 0) {
-          const int y = (bh * G.ntmax + s_idx[t]) * S;
+          const int j = s_idx[t];
           mbar_arrive_expect_tx(bar(BAR_VFULL + st), (uint32_t)C::kTileBytes);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(sV + st * C::kTileBytes + c * BN * 128, &tmV, bar(BAR_VFULL + st), 64 * c, y);
+            load_tile(sV + st * C::kTileBytes + c * BN * 128, tmV, bar(BAR_VFULL + st), c, j);
         }
         __syncwarp();
         issued = t + 1;
@@ -464,7 +493,18 @@ __global__ void __launch_bounds__(384, 1)
       const float inv_l = (l_tot > 0.f) ? 1.0f / l_tot : 0.f;
       const float cA = wA * inv_l, cB = wB * inv_l;
       // stream s writes output columns [s*D/2, (s+1)*D/2), reading both O's
-      const long long grow = ((long long)bh * G.ntmax + i) * S + row;
+      long long grow;
+      bool valid = row < S;
+      if constexpr (GRID) {
+        const int iw = i % hg.nTw, ih = (i / hg.nTw) % hg.nTh, it = i / (hg.nTw * hg.nTh);
+        const int x = iw * hg.pw + row % hg.pw;
+        const int y = ih * hg.ph + (row / hg.pw) % hg.ph;
+        const int tt = it * hg.pt + row / (hg.pw * hg.ph);
+        valid = valid && tt < G.T && y < G.H && x < G.W;
+        grow = (long long)bh * G.N + ((long long)tt * G.H + y) * G.W + x;
+      } else {
+        grow = ((long long)bh * G.ntmax + i) * S + row;
+      }
       uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(A.op) + grow * D + s * (D / 2));
 #pragma unroll
       for (int c = 0; c < D / 2; c += 32) {
@@ -474,7 +514,7 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int q = 0; q < 32; ++q) oa[q] = (cA != 0.f ? cA * oa[q] : 0.f) + (cB != 0.f ? cB * ob[q] : 0.f);
-        if (row < S) {
+        if (valid) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint4 v;
@@ -486,7 +526,7 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
-      if (A.lse != nullptr && s == 0 && row < S)
+      if (A.lse != nullptr && s == 0 && valid)
         A.lse[grow] = (l_tot > 0.f) ? (m + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
     }
   }
@@ -499,32 +539,32 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-template <int D, int BN, int KST, int VST>
-static cudaError_t launch_attn_t(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,
-                                 const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s) {
+template <int D, int BN, int KST, int VST, bool GRID>
+static cudaError_t launch_attn_t(const Geometry& G, const AttnMaps<GRID ? kMaxGridMaps : 1>& m,
+                                 const AttnArgs& a, cudaStream_t s) {
   using C = AttnCfg<D, BN, KST, VST>;
+  auto kernel = sparse_attn_kernel<D, BN, KST, VST, GRID>;
   const size_t smem = C::smem_bytes(a.k_max);
-  cudaError_t err = cudaFuncSetAttribute(sparse_attn_kernel<D, BN, KST, VST>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   // setmaxnreg moves registers between warpgroups inside the block's launch
   // allocation: 128 threads drop to 56 and 256 threads rise to 224.  The
   // split must fit the registers the block is launched with, or the raise
   // would wait forever; refuse to launch otherwise.
   cudaFuncAttributes attr;
-  if ((err = cudaFuncGetAttributes(&attr, sparse_attn_kernel<D, BN, KST, VST>)) != cudaSuccess) return err;
+  if ((err = cudaFuncGetAttributes(&attr, kernel)) != cudaSuccess) return err;
   if (128 * 56 + 256 * 224 > C::kThreads * attr.numRegs) return cudaErrorInvalidConfiguration;
-  const unsigned blocks = (unsigned)(G.B * G.heads * G.ntmax);
-  sparse_attn_kernel<D, BN, KST, VST><<<blocks, C::kThreads, smem, s>>>(tq, tk, tv, G, a);
+  const unsigned blocks = (unsigned)(G.B * (GRID ? a.n_group : G.heads) * G.ntmax);
+  kernel<<<blocks, C::kThreads, smem, s>>>(m, G, a);
   return cudaGetLastError();
 }
 
-template <int D, int BN>
-static cudaError_t launch_attn_d(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,
-                                 const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s) {
+template <int D, int BN, bool GRID>
+static cudaError_t launch_attn_d(const Geometry& G, const AttnMaps<GRID ? kMaxGridMaps : 1>& m,
+                                 const AttnArgs& a, cudaStream_t s) {
   if (AttnCfg<D, BN, 3, 2>::smem_bytes(a.k_max) <= (size_t)kSmemLimit)
-    return launch_attn_t<D, BN, 3, 2>(G, tq, tk, tv, a, s);
-  return launch_attn_t<D, BN, 2, 2>(G, tq, tk, tv, a, s);
+    return launch_attn_t<D, BN, 3, 2, GRID>(G, m, a, s);
+  return launch_attn_t<D, BN, 2, 2, GRID>(G, m, a, s);
 }
 
 size_t sparse_attn_smem_bytes(int d, int S, int k_max) {
@@ -537,10 +577,22 @@ size_t sparse_attn_smem_bytes(int d, int S, int k_max) {
 
 cudaError_t launch_sparse_attn(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s) {
-  if (G.d == 128 && G.S == 128) return launch_attn_d<128, 128>(G, tq, tk, tv, a, s);
-  if (G.d == 128 && G.S == 64) return launch_attn_d<128, 64>(G, tq, tk, tv, a, s);
-  if (G.d == 64 && G.S == 128) return launch_attn_d<64, 128>(G, tq, tk, tv, a, s);
-  return launch_attn_d<64, 64>(G, tq, tk, tv, a, s);
+  AttnMaps<1> m;
+  m.q[0] = tq;
+  m.k[0] = tk;
+  m.v[0] = tv;
+  if (G.d == 128 && G.S == 128) return launch_attn_d<128, 128, false>(G, m, a, s);
+  if (G.d == 128 && G.S == 64) return launch_attn_d<128, 64, false>(G, m, a, s);
+  if (G.d == 64 && G.S == 128) return launch_attn_d<64, 128, false>(G, m, a, s);
+  return launch_attn_d<64, 64, false>(G, m, a, s);
+}
+
+cudaError_t launch_sparse_attn_grid(const Geometry& G, const AttnMaps<kMaxGridMaps>& m, const AttnArgs& a,
+                                    cudaStream_t s) {
+  if (G.d == 128 && G.S == 128) return launch_attn_d<128, 128, true>(G, m, a, s);
+  if (G.d == 128 && G.S == 64) return launch_attn_d<128, 64, true>(G, m, a, s);
+  if (G.d == 64 && G.S == 128) return launch_attn_d<64, 128, true>(G, m, a, s);
+  return launch_attn_d<64, 64, true>(G, m, a, s);
 }
 
 }  // namespace veda

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -137,6 +138,28 @@ veda_status encode_tile_major(const Geometry& G, const void* ptr, CUtensorMap* o
   return VEDA_OK;
 }
 
+// 5D view [B*heads, T, H, W, d] of a grid-order bf16 tensor [B, heads, N, d]
+// with boxes of 64 channels x pw x ph x pt tokens x 1: one box is one 3D tile
+// of a head with tiling (pt, ph, pw), in within-tile slot order.  Boxes that
+// reach past the grid are zero-filled.  128-byte swizzle as above.
+veda_status encode_grid_tiles(const Geometry& G, const void* ptr, const HeadGeom& hg, CUtensorMap* out) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t row = (cuuint64_t)G.d * 2;
+  const cuuint64_t dims[5] = {(cuuint64_t)G.d, (cuuint64_t)G.W, (cuuint64_t)G.H, (cuuint64_t)G.T,
+                              (cuuint64_t)G.B * G.heads};
+  const cuuint64_t strides[4] = {row, row * G.W, row * G.W * G.H, row * (cuuint64_t)G.N};
+  const cuuint32_t box[5] = {64u, (cuuint32_t)hg.pw, (cuuint32_t)hg.ph, (cuuint32_t)hg.pt, 1u};
+  const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+  const CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled (grid tiles %dx%dx%d) failed (CUresult %d)", hg.pt, hg.ph,
+                hg.pw, (int)r);
+  return VEDA_OK;
+}
+
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 size_t score_ws_bytes(const Geometry& G, int e) {
@@ -237,6 +260,17 @@ veda_status veda_tripool(const veda_problem* p, const void* xp, float* desc, voi
   if (!aligned16(xp) || !aligned16(desc)) return fail(VEDA_ERR_INVALID_ARG, "xp and desc must be 16-byte aligned");
   cudaError_t e = launch_tripool(G, xp, desc, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "veda_tripool");
+  return ok();
+}
+
+veda_status veda_tripool_grid(const veda_problem* p, const void* x, float* desc, void* stream) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (!x || !desc) return fail(VEDA_ERR_INVALID_ARG, "x and desc must be non-NULL");
+  if (!aligned16(x) || !aligned16(desc)) return fail(VEDA_ERR_INVALID_ARG, "x and desc must be 16-byte aligned");
+  cudaError_t e = launch_tripool_grid(G, x, desc, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "veda_tripool_grid");
   return ok();
 }
 
@@ -402,6 +436,7 @@ veda_status veda_tile_sparse_attn(const veda_problem* p, const void* qp, const v
       (s = encode_tile_major(G, vp, &tv)) != VEDA_OK)
     return s;
   AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
   a.idx = idx;
   a.k_max = k_max;
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)G.d);
@@ -411,6 +446,67 @@ veda_status veda_tile_sparse_attn(const veda_problem* p, const void* qp, const v
   a.timeout_ns = g_timeout_ns;
   cudaError_t e = launch_sparse_attn(G, tq, tk, tv, a, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "veda_tile_sparse_attn");
+  return ok();
+}
+
+veda_status veda_tile_sparse_attn_grid(const veda_problem* p, const void* q, const void* k, const void* v,
+                                       const int32_t* idx, int32_t k_max, float scale, void* o, float* lse,
+                                       void* stream) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (!q || !k || !v || !idx || !o) return fail(VEDA_ERR_INVALID_ARG, "NULL tensor argument");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(idx) ||
+      (lse && !aligned16(lse)))
+    return fail(VEDA_ERR_INVALID_ARG, "tensor arguments must be 16-byte aligned");
+  if (k_max < 1) return fail(VEDA_ERR_INVALID_ARG, "k_max must be >= 1 (got %d)", k_max);
+  if (!(std::isfinite(scale))) return fail(VEDA_ERR_INVALID_ARG, "scale must be finite");
+  if (sparse_attn_smem_bytes(G.d, G.S, k_max) > 227 * 1024)
+    return fail(VEDA_ERR_UNSUPPORTED, "k_max = %d exceeds the shared-memory budget", k_max);
+  if (G.ntmax > 32767) return fail(VEDA_ERR_UNSUPPORTED, "NT_max = %d exceeds 32767 tiles per head", G.ntmax);
+  // Distinct tilings in order of first appearance; a launch covers up to
+  // kMaxGridMaps of them (one set of tensor maps each).
+  int tiling_of_head[VEDA_MAX_HEADS];
+  int distinct[VEDA_MAX_HEADS];
+  int n_distinct = 0;
+  for (int h = 0; h < G.heads; ++h) {
+    int u = 0;
+    while (u < n_distinct && !(G.g[distinct[u]].pt == G.g[h].pt && G.g[distinct[u]].ph == G.g[h].ph &&
+                               G.g[distinct[u]].pw == G.g[h].pw))
+      ++u;
+    if (u == n_distinct) distinct[n_distinct++] = h;
+    tiling_of_head[h] = u;
+  }
+  AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.idx = idx;
+  a.k_max = k_max;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)G.d);
+  a.scale_log2 = sc * 1.4426950408889634f;
+  a.op = o;
+  a.lse = lse;
+  a.timeout_ns = g_timeout_ns;
+  AttnMaps<kMaxGridMaps> maps;  // copied into the kernel parameters at launch
+  std::memset(&maps, 0, sizeof(maps));
+  for (int u0 = 0; u0 < n_distinct; u0 += kMaxGridMaps) {
+    const int nu = std::min(kMaxGridMaps, n_distinct - u0);
+    for (int u = 0; u < nu; ++u) {
+      const HeadGeom& hg = G.g[distinct[u0 + u]];
+      if ((s = encode_grid_tiles(G, q, hg, &maps.q[u])) != VEDA_OK ||
+          (s = encode_grid_tiles(G, k, hg, &maps.k[u])) != VEDA_OK ||
+          (s = encode_grid_tiles(G, v, hg, &maps.v[u])) != VEDA_OK)
+        return s;
+    }
+    a.n_group = 0;
+    for (int h = 0; h < G.heads; ++h) {
+      const int u = tiling_of_head[h] - u0;
+      if (u < 0 || u >= nu) continue;
+      a.head_list[a.n_group++] = (int16_t)h;
+      a.map_of_head[h] = (int8_t)u;
+    }
+    cudaError_t e = launch_sparse_attn_grid(G, maps, a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "veda_tile_sparse_attn_grid");
+  }
   return ok();
 }
 
