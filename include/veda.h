@@ -214,6 +214,14 @@ veda_status veda_tile_sparse_attn_grid(const veda_problem* p, const void* q, con
                                        const void* v, const int32_t* idx, int32_t k_max, float scale,
                                        void* o, float* lse, void* stream);
 
+/* Launch configuration the two attention calls use for this problem and
+ * k_max (host-side query, no device work): the depths of the K and V tile
+ * rings in shared memory and the dynamic shared memory per CTA.  Deeper
+ * rings are chosen whenever they fit; the bookkeeping (selection list) grows
+ * with k_max.  Returns VEDA_ERR_UNSUPPORTED when no configuration fits. */
+veda_status veda_attn_config(const veda_problem* p, int32_t k_max, int32_t* k_stages, int32_t* v_stages,
+                             size_t* smem_bytes);
+
 /* ---------------------------------------------------------------- secondary: tile map */
 
 /* Bytes of workspace veda_tile_map_maxpool needs for R subset rows. */

@@ -108,3 +108,18 @@ def test_workspace_sizes(V):
     assert V.veda_tile_map_workspace(p, R) >= 4 * 2 * 3 * R * (p.nt_max * 64 + 64)
     with pytest.raises(V.VedaError):
         V.veda_score_topk_workspace(p, 3)
+
+
+def test_attention_config_query(V):
+    """Ring depths and shared memory of the attention launch, computed on the host."""
+    p = V.Problem(1, 2, 128, 128, (21, 45, 80), [(2, 8, 8), (8, 4, 4)])
+    ks, vs, smem = V.veda_attn_config(p, 36)
+    assert (ks, vs) == (3, 3) and smem <= 232448
+    # a long selection list grows the bookkeeping past the 3/3 budget
+    ks, vs, smem2 = V.veda_attn_config(p, 400)
+    assert (ks, vs) == (3, 2) and smem2 <= 232448
+    # 16 KB tiles (d = 64) take four stages of each
+    p64 = V.Problem(1, 1, 64, 64, (4, 8, 8), [(1, 8, 8)])
+    assert V.veda_attn_config(p64, 2)[:2] == (4, 4)
+    with pytest.raises(V.VedaError):
+        V.veda_attn_config(p, 0)

@@ -66,6 +66,7 @@ _SIG = {
                                      _V, ctypes.c_int32, _V, _V],
     "veda_tile_sparse_attn": [_P, _V, _V, _V, _V, ctypes.c_int32, ctypes.c_float, _V, _V, _V],
     "veda_tile_sparse_attn_grid": [_P, _V, _V, _V, _V, ctypes.c_int32, ctypes.c_float, _V, _V, _V],
+    "veda_attn_config": [_P, ctypes.c_int32, _I32P, _I32P, ctypes.POINTER(ctypes.c_size_t)],
     "veda_tile_map_workspace": [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)],
     "veda_tile_map_maxpool": [_P, _V, _V, _V, ctypes.c_int32, ctypes.c_float, _V, _V, ctypes.c_size_t, _V],
     "veda_sync_status": [_V],
@@ -271,6 +272,14 @@ def veda_tile_sparse_attn_grid(p: Problem, q: torch.Tensor, k: torch.Tensor, v: 
         _ptr(lse, "lse", torch.float32, (p.B, p.heads, p.N)), _stream(stream)),
         "veda_tile_sparse_attn_grid")
     return o
+
+
+def veda_attn_config(p: Problem, k_max: int) -> Tuple[int, int, int]:
+    """(K ring depth, V ring depth, dynamic shared memory bytes) of the attention launch."""
+    ks, vs, nb = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_size_t()
+    _check(LIB.veda_attn_config(p.ref, int(k_max), ctypes.byref(ks), ctypes.byref(vs), ctypes.byref(nb)),
+           "veda_attn_config")
+    return int(ks.value), int(vs.value), int(nb.value)
 
 
 def veda_tile_map_workspace(p: Problem, R: int) -> int:

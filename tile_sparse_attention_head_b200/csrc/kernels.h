@@ -70,6 +70,8 @@ cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const floa
                               const EstimatorWeights& wq, const EstimatorWeights& wk, int hidden,
                               int e, float* phi, const TopkArgs& args, cudaStream_t s);
 
+size_t sparse_attn_smem_bytes(int d, int S, int k_max);
+void sparse_attn_config(int d, int S, int k_max, int* k_stages, int* v_stages, size_t* smem);
 cudaError_t launch_sparse_attn(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tv, const AttnArgs& a, cudaStream_t s);
 // Grid-order variant: Q/K/V tiles are fetched as 5D boxes of the grid-order

@@ -40,11 +40,16 @@
 
 namespace veda {
 
-// One exponential in kPolyEvery is evaluated with exp2_fma (FMA pipe), the
-// others with ex2.approx (special-function unit), balancing the two pipes.
-constexpr int kPolyEvery = 4;
+// Three pairs of exponentials in eight are evaluated with exp2_fma_x2 (FMA
+// pipe), the others with ex2.approx (special-function unit, a quarter of the
+// FMA rate): this balances the two pipes of a row of 128 scores.
+__host__ __device__ constexpr bool poly_pair(int pair) { return (pair * 3) % 8 < 3; }
 constexpr int kSmemLimit = 232448;   // dynamic shared memory per CTA on sm_100
 
+// Shared memory: the bookkeeping (barriers, the final (m, l) exchange, flags,
+// the selection list) first, then -- from the next 1024-byte boundary, as the
+// 128-byte swizzle needs -- the operand region Q | K ring | V ring.  The
+// dynamic shared memory base must itself be 1024-byte aligned (checked).
 template <int D, int BN, int KST, int VST>
 struct AttnCfg {
   static constexpr int BM = 128;                 // MMA rows (query slots; S = 64 tiles use half)
@@ -52,19 +57,24 @@ struct AttnCfg {
   static constexpr int kChunk = 128 * 128;       // one [128 rows x 128 B] swizzle panel
   static constexpr int kQBytes = BM * D * 2;
   static constexpr int kTileBytes = BN * D * 2;  // one K or V tile
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + KST * kTileBytes;
-  static constexpr int kOffBar = kOffV + VST * kTileBytes;
+  static constexpr int kOffBar = 0;
   static constexpr int kNumBars = 32;
   static constexpr int kOffRed = kOffBar + kNumBars * 8;   // float [2 stream][2: m, l][128 rows]
   static constexpr int kOffMisc = kOffRed + 2 * 2 * 128 * 4;
-  static constexpr int kOffIdx = kOffMisc + 64;
+  static constexpr int kOffIdx = kOffMisc + 64;  // int16 selection list, then int32 valid extents
+  // offsets inside the operand region
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffV = kOffK + KST * kTileBytes;
+  static constexpr int kOperandBytes = kOffV + VST * kTileBytes;
+  __host__ __device__ static size_t bookkeeping_bytes(int k_max) {
+    return (kOffIdx + 6 * (size_t)((k_max + 7) & ~7) + 1023) & ~size_t(1023);
+  }
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemS = 0;          // S, shared by the streams
   static constexpr uint32_t kTmemP = 128;        // P of stream s at kTmemP + 64 s (packed bf16)
   static constexpr uint32_t kTmemO = 256;        // O of stream s at kTmemO + 128 s
-  static size_t smem_bytes(int k_max) { return 1024 + kOffIdx + 2 * (size_t)((k_max + 7) & ~7); }
+  static size_t smem_bytes(int k_max) { return bookkeeping_bytes(k_max) + kOperandBytes; }
 };
 
 // mbarrier slots
@@ -132,8 +142,12 @@ __global__ void __launch_bounds__(384, 1)
     sparse_attn_kernel(const __grid_constant__ AttnMaps<GRID ? kMaxGridMaps : 1> M,
                        const __grid_constant__ Geometry G, const __grid_constant__ AttnArgs A) {
   using C = AttnCfg<D, BN, KST, VST>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {   // CTA-uniform, before any barrier or TMEM use
+    if (threadIdx.x == 0) atomicExch(&g_device_error, kErrSmemAlign);
+    return;
+  }
+  uint8_t* ops = smem + C::bookkeeping_bytes(A.k_max);   // operand region, 1024-byte aligned
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int i = blockIdx.x % G.ntmax;
@@ -163,14 +177,17 @@ __global__ void __launch_bounds__(384, 1)
     }
   };
 
-  const uint32_t sQ = smem_u32(smem + C::kOffQ);
-  const uint32_t sK = smem_u32(smem + C::kOffK);
-  const uint32_t sV = smem_u32(smem + C::kOffV);
+  const uint32_t sQ = smem_u32(ops + C::kOffQ);
+  const uint32_t sK = smem_u32(ops + C::kOffK);
+  const uint32_t sV = smem_u32(ops + C::kOffV);
   const uint32_t bar0 = smem_u32(smem + C::kOffBar);
   auto bar = [&](int b) { return bar0 + 8u * (uint32_t)b; };
   float* red = reinterpret_cast<float*>(smem + C::kOffRed);
   int* misc = reinterpret_cast<int*>(smem + C::kOffMisc);  // [0] tmem base, [1] abort, [2] n_sel
   int16_t* s_idx = reinterpret_cast<int16_t*>(smem + C::kOffIdx);
+  // valid extents (ct | ch << 8 | cw << 16) of each selected tile, bit 24 set
+  // when the tile has pad slots (an edge tile)
+  uint32_t* s_ext = reinterpret_cast<uint32_t*>(smem + C::kOffIdx + 2 * ((A.k_max + 7) & ~7));
   volatile int* abort = misc + 1;
 
   if (tid == 0) {
@@ -182,7 +199,15 @@ __global__ void __launch_bounds__(384, 1)
   for (int c = tid; c < A.k_max; c += C::kThreads) {
     const int v = irow[c];
     s_idx[c] = (int16_t)v;
-    if (v < 0 || v >= hg.nt) atomicMin(&misc[2], c);  // the list ends at the first invalid entry
+    if (v < 0 || v >= hg.nt) {
+      atomicMin(&misc[2], c);  // the list ends at the first invalid entry
+      continue;
+    }
+    const int jw = v % hg.nTw, jh = (v / hg.nTw) % hg.nTh, jt = v / (hg.nTw * hg.nTh);
+    const int ct = min((int)hg.pt, G.T - jt * hg.pt);
+    const int ch = min((int)hg.ph, G.H - jh * hg.ph);
+    const int cw = min((int)hg.pw, G.W - jw * hg.pw);
+    s_ext[c] = (uint32_t)ct | ((uint32_t)ch << 8) | ((uint32_t)cw << 16) | (ct * ch * cw != S ? 1u << 24 : 0u);
   }
   if (tid == 0) {
     mbar_init(bar(BAR_Q), 1);
@@ -212,7 +237,7 @@ __global__ void __launch_bounds__(384, 1)
   if (BN < 128 && warp >= 4) {
     // S = 64: the MMA always runs 128 rows; rows 64..127 of the Q panels are zero.
     for (int c = 0; c < D / 64; ++c) {
-      uint4* p = reinterpret_cast<uint4*>(smem + C::kOffQ + c * C::kChunk + 64 * 128);
+      uint4* p = reinterpret_cast<uint4*>(ops + C::kOffQ + c * C::kChunk + 64 * 128);
       for (int e = tid - 128; e < 64 * 128 / 16; e += 256) p[e] = make_uint4(0, 0, 0, 0);
     }
     fence_proxy_async_smem();
@@ -381,12 +406,9 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0) mbar_arrive(bar(BAR_SFREE + s));
 
       // Pad keys of an edge tile are masked out.
-      const int j = s_idx[t];
-      const int jw = j % hg.nTw, jh = (j / hg.nTw) % hg.nTh, jt = j / (hg.nTw * hg.nTh);
-      const int ct = min((int)hg.pt, G.T - jt * hg.pt);
-      const int ch = min((int)hg.ph, G.H - jh * hg.ph);
-      const int cw = min((int)hg.pw, G.W - jw * hg.pw);
-      if (ct * ch * cw != S) {
+      const uint32_t ext = s_ext[t];
+      if (ext >> 24) {
+        const int ct = (int)(ext & 255u), ch = (int)((ext >> 8) & 255u), cw = (int)((ext >> 16) & 255u);
         uint32_t mw[BN / 32];
 #pragma unroll
         for (int w = 0; w < BN / 32; ++w) mw[w] = __ballot_sync(0xffffffffu, kt[w] < ct && ky[w] < ch && kx[w] < cw);
@@ -429,7 +451,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int c = 0; c < BN; c += 2) {
         float x0, x1, p0, p1;
         f2_split(f2_fma(f2(sc[c], sc[c + 1]), scl2, nref2), x0, x1);
-        if ((c >> 1) % kPolyEvery == kPolyEvery - 1) {
+        if (poly_pair(c >> 1)) {
           exp2_fma_x2(x0, x1, p0, p1);
         } else {
           p0 = fast_exp2(x0);
@@ -559,12 +581,55 @@ static cudaError_t launch_attn_t(const Geometry& G, const AttnMaps<GRID ? kMaxGr
   return cudaGetLastError();
 }
 
+// The deepest K/V rings that fit: a K/V tile fetch from L2 takes a few
+// thousand cycles under load, and the V ring in particular is refilled only
+// after the PV product that read its stage, so ring depth sets the tile rate.
+template <int D, int BN>
+static int attn_stages_t(int k_max) {   // returns 10 * K stages + V stages
+  if (D * BN <= 64 * 128 && AttnCfg<D, BN, 4, 4>::smem_bytes(k_max) <= (size_t)kSmemLimit) return 44;
+  if (AttnCfg<D, BN, 3, 3>::smem_bytes(k_max) <= (size_t)kSmemLimit) return 33;
+  if (AttnCfg<D, BN, 3, 2>::smem_bytes(k_max) <= (size_t)kSmemLimit) return 32;
+  return 22;
+}
+
 template <int D, int BN, bool GRID>
 static cudaError_t launch_attn_d(const Geometry& G, const AttnMaps<GRID ? kMaxGridMaps : 1>& m,
                                  const AttnArgs& a, cudaStream_t s) {
-  if (AttnCfg<D, BN, 3, 2>::smem_bytes(a.k_max) <= (size_t)kSmemLimit)
-    return launch_attn_t<D, BN, 3, 2, GRID>(G, m, a, s);
-  return launch_attn_t<D, BN, 2, 2, GRID>(G, m, a, s);
+  switch (attn_stages_t<D, BN>(a.k_max)) {
+    case 44:
+      if constexpr (D * BN <= 64 * 128) return launch_attn_t<D, BN, 4, 4, GRID>(G, m, a, s);
+      return cudaErrorInvalidConfiguration;
+    case 33: return launch_attn_t<D, BN, 3, 3, GRID>(G, m, a, s);
+    case 32: return launch_attn_t<D, BN, 3, 2, GRID>(G, m, a, s);
+    default: return launch_attn_t<D, BN, 2, 2, GRID>(G, m, a, s);
+  }
+}
+
+// K and V ring depths and dynamic shared memory the attention launch uses.
+void sparse_attn_config(int d, int S, int k_max, int* k_stages, int* v_stages, size_t* smem) {
+  int ks = 22;
+  size_t bytes = 0;
+  auto pick = [&](auto cfg44, auto cfg33, auto cfg32, auto cfg22, int code) {
+    ks = code;
+    bytes = code == 44 ? decltype(cfg44)::smem_bytes(k_max)
+          : code == 33 ? decltype(cfg33)::smem_bytes(k_max)
+          : code == 32 ? decltype(cfg32)::smem_bytes(k_max) : decltype(cfg22)::smem_bytes(k_max);
+  };
+  if (d == 128 && S == 128)
+    pick(AttnCfg<128, 128, 4, 4>{}, AttnCfg<128, 128, 3, 3>{}, AttnCfg<128, 128, 3, 2>{}, AttnCfg<128, 128, 2, 2>{},
+         attn_stages_t<128, 128>(k_max));
+  else if (d == 128)
+    pick(AttnCfg<128, 64, 4, 4>{}, AttnCfg<128, 64, 3, 3>{}, AttnCfg<128, 64, 3, 2>{}, AttnCfg<128, 64, 2, 2>{},
+         attn_stages_t<128, 64>(k_max));
+  else if (S == 128)
+    pick(AttnCfg<64, 128, 4, 4>{}, AttnCfg<64, 128, 3, 3>{}, AttnCfg<64, 128, 3, 2>{}, AttnCfg<64, 128, 2, 2>{},
+         attn_stages_t<64, 128>(k_max));
+  else
+    pick(AttnCfg<64, 64, 4, 4>{}, AttnCfg<64, 64, 3, 3>{}, AttnCfg<64, 64, 3, 2>{}, AttnCfg<64, 64, 2, 2>{},
+         attn_stages_t<64, 64>(k_max));
+  *k_stages = ks / 10;
+  *v_stages = ks % 10;
+  *smem = bytes;
 }
 
 size_t sparse_attn_smem_bytes(int d, int S, int k_max) {

@@ -510,6 +510,24 @@ veda_status veda_tile_sparse_attn_grid(const veda_problem* p, const void* q, con
   return ok();
 }
 
+veda_status veda_attn_config(const veda_problem* p, int32_t k_max, int32_t* k_stages, int32_t* v_stages,
+                             size_t* smem_bytes) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (k_max < 1) return fail(VEDA_ERR_INVALID_ARG, "k_max must be >= 1 (got %d)", k_max);
+  if (!k_stages || !v_stages || !smem_bytes) return fail(VEDA_ERR_INVALID_ARG, "NULL output argument");
+  if (sparse_attn_smem_bytes(G.d, G.S, k_max) > 227 * 1024)
+    return fail(VEDA_ERR_UNSUPPORTED, "k_max = %d exceeds the shared-memory budget", k_max);
+  int ks = 0, vs = 0;
+  size_t bytes = 0;
+  sparse_attn_config(G.d, G.S, k_max, &ks, &vs, &bytes);
+  *k_stages = ks;
+  *v_stages = vs;
+  *smem_bytes = bytes;
+  return ok();
+}
+
 veda_status veda_tile_map_workspace(const veda_problem* p, int32_t R, size_t* bytes) {
   Geometry G;
   veda_status s = make_geometry(p, &G);
@@ -560,6 +578,8 @@ veda_status veda_sync_status(void* stream) {
   if (word != kErrNone) {
     const int zero = 0;
     cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+    if (word == kErrSmemAlign)
+      return fail(VEDA_ERR_CUDA, "a kernel found its dynamic shared memory base not 1024-byte aligned");
     return fail(VEDA_ERR_TIMEOUT, "a kernel gave up on a bounded wait (device error word %d)", word);
   }
   return ok();

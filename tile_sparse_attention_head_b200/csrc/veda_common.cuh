@@ -70,7 +70,7 @@ __device__ __forceinline__ int tile_token_count(const Geometry& G, const HeadGeo
 // Device error word: kernels that give up on a bounded wait record a code here
 // and return; veda_sync_status() reads and clears it.
 // ----------------------------------------------------------------------------
-enum : int { kErrNone = 0, kErrTimeout = 1 };
+enum : int { kErrNone = 0, kErrTimeout = 1, kErrSmemAlign = 2 };
 __device__ int g_device_error = 0;
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -385,6 +385,11 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -392,25 +397,22 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 }
 
 // exp2_fma on a pair of lanes: the reduction and the cubic run as packed
-// f32x2 operations, the exponent insertion per lane.
+// f32x2 operations, the exponent insertion per lane.  With t = x + 1.5*2^23
+// the bits of t are 0x4B400000 + j, and 0x4B400000 << 23 vanishes modulo
+// 2^32, so adding bits(t) << 23 to the cubic's bits adds j to its exponent.
 __device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& y0, float& y1) {
-  x0 = fmaxf(x0, -126.0f);
-  x1 = fmaxf(x1, -126.0f);
-  const uint64_t x = f2(x0, x1);
+  const uint64_t x = f2(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
   const uint64_t magic = f2(12582912.0f, 12582912.0f);
-  const uint64_t nmagic = f2(-12582912.0f, -12582912.0f);
   const uint64_t t = f2_add(x, magic);
-  float r0, r1, t0, t1;
-  f2_split(f2_add(t, nmagic), r0, r1);
-  const uint64_t f = f2_add(x, f2(-r0, -r1));
+  const uint64_t f = f2_sub(x, f2_sub(t, magic));
   uint64_t p = f2_fma(f2(0.0551716685f, 0.0551716685f), f, f2(0.2426111251f, 0.2426111251f));
   p = f2_fma(p, f, f2(0.6932609677f, 0.6932609677f));
   p = f2_fma(p, f, f2(0.9999280572f, 0.9999280572f));
-  float p0, p1;
+  float p0, p1, t0, t1;
   f2_split(p, p0, p1);
   f2_split(t, t0, t1);
-  y0 = __int_as_float(__float_as_int(p0) + ((__float_as_int(t0) - 0x4B400000) << 23));
-  y1 = __int_as_float(__float_as_int(p1) + ((__float_as_int(t1) - 0x4B400000) << 23));
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
