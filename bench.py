@@ -52,10 +52,11 @@ WORKLOAD_NAMES = {"wan14b": "Wan2.1-14B-720p-81f 21x45x80 (75,600 tokens) 40 hea
 
 
 # DRAM bytes (read + write) of one attention launch, from a one-pass ncu
-# capture of the benchmarked launch (profiles/sparse_attn_wan14b.md), keyed by
-# workload and tied to the kernel source it was measured on: reported only
-# while csrc/sparse_attn.cu still hashes to that version.
-ATTN_TRAFFIC = {("wan14b", "tile"): {"bytes": 1.26e9 + 858.49e6, "src_sha256_16": "b5a8f826b6c7f91f"}}
+# capture of the benchmarked launch (summarised with the committed profiles),
+# keyed by workload and layout and tied to the kernel source it was measured
+# on: reported only while csrc/sparse_attn.cu still hashes to that version.
+ATTN_TRAFFIC = {("wan14b", "tile"): {"bytes": 1.26e9 + 858.49e6, "src_sha256_16": "b5a8f826b6c7f91f"},
+                ("wan14b", "grid"): {"bytes": 1.16e9 + 740.09e6, "src_sha256_16": "46d3959bdaeadfc5"}}
 
 
 def attn_traffic(workload: str, layout: str):
