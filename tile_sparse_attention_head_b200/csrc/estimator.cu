@@ -1,176 +1,289 @@
 // Head-specific MLP estimator (section 2.1 of the Veda summary: a separate
 // MLP projection per attention head maps each tile's TripPool descriptor
 // into the space where tile scores are formed):
-//     phi = W2 relu(W1 desc + b1) + b2,   fp32.
+//     phi = W2 relu(W1 desc + b1) + b2,   fp32 in, fp32 out.
 //
-// Per (head, Q-or-K side) this is two small GEMMs, [NT x 3d] x [3d x hidden]
-// and [NT x hidden] x [hidden x e].  They stay in fp32 on the CUDA cores
-// (tile selection is decided on these values, so they must not be rounded to
-// a tensor-core input type): one CTA takes 64 tiles, stages 32-wide k panels
-// of both operands k-major in shared memory, and every thread accumulates a
-// 4 x 4 register block, so each pair of 16-byte shared loads feeds 16 FMAs.
-// The hidden activations stay in shared memory for the second GEMM.
+// Per (head, Q-or-K side) this is two dense contractions,
+// [NT x 3d] x [3d x hidden] and [NT x hidden] x [hidden x e], so it runs on
+// the sm_100a tensor cores (tcgen05, kind::tf32, accumulators in TMEM).
+// Tile selection is decided on these values, so they keep fp32 accuracy:
+// every operand is split as x = hi + lo (hi the nearest tf32 value, lo the
+// exact fp32 remainder) and each product is formed as hi*hi + hi*lo + lo*hi,
+// which carries it to about 2^-21 relative (the dropped lo*lo term is below
+// that).
+//
+// One CTA takes 128 tiles (the MMA's M) of one (b, h, side).  The hidden
+// layer is produced in passes of up to 256 units (the MMA's N):
+//   layer 1: 32-wide k panels of the descriptor and of W1 are loaded by all
+//     256 threads, split, and written 128-byte-swizzled (K-major) into one
+//     of two shared-memory stages while the MMAs of the previous panel run;
+//     one thread issues 4 k-steps x 3 products per panel into TMEM.
+//   layer 2: for every 32 hidden units, warps 0-3 read the layer-1
+//     accumulator from TMEM (one tile row per thread), add b1, apply ReLU and
+//     split; warps 4-7 stage the matching 32 columns of W2; the products
+//     accumulate phi in a second TMEM region across all passes.
+// Finally warps 0-3 add b2 and store phi.  Waits are bounded; the whole CTA
+// agrees on an abort at every barrier (a predicate-reducing __syncthreads),
+// so no thread is left behind at a barrier, and all MMAs are drained before
+// TMEM is freed.
 #pragma once
 #include "veda_common.cuh"
 #include "kernels.h"
 
 namespace veda {
 
-constexpr int kEstRows = 64;     // tiles per CTA
-constexpr int kEstK = 32;        // k panel width
-constexpr int kEstLd = 68;       // shared row stride (floats) of 64-wide k-major panels
-
-__host__ __device__ inline int est_ws_ld(int e) { return (e + 4) > kEstLd ? (e + 4) : kEstLd; }
+constexpr int kEstRows = 128;                       // tiles per CTA (MMA M)
+constexpr int kEstThreads = 256;
+constexpr int kEstN1 = 256;                         // hidden units per layer-1 pass (MMA N)
+constexpr int kEstPanelA = 128 * 128;               // 128 rows x 32 fp32
+constexpr int kEstPanelB = 256 * 128;               // up to 256 rows x 32 fp32
+constexpr int kEstStage = 2 * kEstPanelA + 2 * kEstPanelB;   // A hi/lo, B hi/lo: 96 KB
+constexpr uint32_t kEstTmemCols = 512;
+constexpr uint32_t kEstAcc1 = 0;                    // layer-1 accumulator, up to 256 columns
+constexpr uint32_t kEstAcc2 = 256;                  // phi accumulator, e <= 128 columns
 
 size_t estimator_smem_bytes(int d, int hidden, int e) {
   (void)d;
-  const int hid_pad = (hidden + 63) / 64 * 64;
-  return sizeof(float) * ((size_t)kEstK * kEstLd + (size_t)kEstK * est_ws_ld(e) + (size_t)hid_pad * kEstLd);
+  (void)hidden;
+  (void)e;
+  return 1024 + 2 * (size_t)kEstStage + 4 * 8 + 16;
 }
 
-// grid: (ceil(NT_max / 64), B*heads, 2); z = 0 -> Q descriptors, z = 1 -> K.
-// CW = e / 16 output columns per thread in the second GEMM.
-template <int CW>
-__global__ void __launch_bounds__(256)
+// Address of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled, K-major
+// panel whose base is 1024-byte aligned.
+__device__ __forceinline__ uint8_t* sw128_chunk(uint8_t* panel, int r, int c) {
+  return panel + r * 128 + ((c ^ (r & 7)) << 4);
+}
+
+__device__ __forceinline__ void store_split4(uint8_t* hi_panel, uint8_t* lo_panel, int r, int c, float4 v) {
+  float4 h, l;
+  split_tf32(v.x, h.x, l.x);
+  split_tf32(v.y, h.y, l.y);
+  split_tf32(v.z, h.z, l.z);
+  split_tf32(v.w, h.w, l.w);
+  *reinterpret_cast<float4*>(sw128_chunk(hi_panel, r, c)) = h;
+  *reinterpret_cast<float4*>(sw128_chunk(lo_panel, r, c)) = l;
+}
+
+// grid: (ceil(NT_max / 128), B*heads, 2); z = 0 -> Q descriptors, z = 1 -> K.
+template <int E>
+__global__ void __launch_bounds__(kEstThreads, 1)
     estimator_kernel(const __grid_constant__ Geometry G, const float* __restrict__ desc_q,
                      const float* __restrict__ desc_k, EstimatorWeights wq, EstimatorWeights wk, int hidden,
-                     float* __restrict__ phi) {
-  constexpr int E = 16 * CW;
-  extern __shared__ float sm[];
-  const int ws_ld = est_ws_ld(E);
-  float* xs = sm;                       // [32][68]     descriptor panel, k-major
-  float* ws = xs + kEstK * kEstLd;      // [32][ws_ld]  W1 panel (64 units) / W2 panel (e outputs)
-  float* hs = ws + kEstK * ws_ld;       // [hid][68]    relu(hidden), k-major
+                     float* __restrict__ phi, uint64_t timeout_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kEstStage);   // [0,1] stage free, [2] layer done, [3] drain
+  int* misc = reinterpret_cast<int*>(bars + 4);                          // [0] TMEM base, [1] abort
 
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int which = blockIdx.z;
   const int bh = blockIdx.y;
   const int h = bh % G.heads;
   const int nt = G.g[h].nt;
   const int j0 = blockIdx.x * kEstRows;
-  if (j0 >= nt) return;
+  if (j0 >= nt) return;   // CTA-uniform, before any barrier or TMEM use
   const int nrows = min(kEstRows, nt - j0);
-  const int in_dim = 3 * G.d;
+  const int K1 = 3 * G.d;
   const EstimatorWeights& w = which ? wk : wq;
-  const float* X = (which ? desc_k : desc_q) + ((long long)bh * G.ntmax + j0) * in_dim;
-  const float* W1 = w.w1 + (long long)h * hidden * in_dim;
+  const float* X = (which ? desc_k : desc_q) + ((long long)bh * G.ntmax + j0) * K1;
+  const float* W1 = w.w1 + (long long)h * hidden * K1;
   const float* B1 = w.b1 + (long long)h * hidden;
   const float* W2 = w.w2 + (long long)h * E * hidden;
   const float* B2 = w.b2 + (long long)h * E;
 
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  const int lr = tid & 63, lk = (tid >> 6) * 4;   // loader: row / unit, k offset (plus 16 on the second half)
+  if (tid == 0) {
+    for (int b = 0; b < 4; ++b) mbar_init(smem_u32(&bars[b]), 1);
+    misc[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&misc[0]), kEstTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+  volatile int* abort = misc + 1;
 
-  // ---- layer 1: hidden = relu(X W1^T + b1), 64 units at a time
-  for (int nb = 0; nb < hidden; nb += 64) {
-    float acc[4][4];
+  int use = 0;     // shared-memory stage uses so far; use u takes stage u & 1
+  int done_phase = 0;
+  bool acc2_started = false;
+  bool ok = true;
+  // Stage (u & 1) is free once the MMAs of use u - 2 have completed.
+  auto wait_stage = [&](int u) -> bool {
+    if (u < 2) return true;
+    return mbar_wait(smem_u32(&bars[u & 1]), ((u - 2) >> 1) & 1, abort, timeout_ns);
+  };
+  auto stage = [&](int u) { return smem + (u & 1) * kEstStage; };
+
+  for (int n0 = 0; ok && n0 < hidden; n0 += kEstN1) {
+    const int n1 = min(kEstN1, hidden - n0);
+    const int n1p = (n1 + 15) & ~15;
+    // ------------------------------------------------------------ layer 1
+    for (int kc = 0; kc < K1 / 32; ++kc) {
+      // descriptor panel: thread -> row tid/2, chunks 4*(tid&1) .. +3
+      // W1 panel: thread -> hidden unit n0 + tid, all 8 chunks
+      float4 xv[4], wv[8];
+      const int xr = tid >> 1, xc = (tid & 1) * 4;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+      for (int q = 0; q < 4; ++q)
+        xv[q] = (xr < nrows) ? __ldg(reinterpret_cast<const float4*>(X + (long long)xr * K1 + kc * 32) + xc + q)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-    for (int k0 = 0; k0 < in_dim; k0 += kEstK) {
-      __syncthreads();
+      for (int q = 0; q < 8; ++q)
+        wv[q] = (tid < n1) ? __ldg(reinterpret_cast<const float4*>(W1 + (long long)(n0 + tid) * K1 + kc * 32) + q)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+      ok = wait_stage(use) && ok;
+      uint8_t* st = stage(use);
+      uint8_t *ahi = st, *alo = st + kEstPanelA, *bhi = st + 2 * kEstPanelA, *blo = bhi + kEstPanelB;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int kq = lk + half * 16;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f), u = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (lr < nrows) v = *reinterpret_cast<const float4*>(X + (long long)lr * in_dim + k0 + kq);
-        if (nb + lr < hidden) u = *reinterpret_cast<const float4*>(W1 + (long long)(nb + lr) * in_dim + k0 + kq);
-        xs[(kq + 0) * kEstLd + lr] = v.x;
-        xs[(kq + 1) * kEstLd + lr] = v.y;
-        xs[(kq + 2) * kEstLd + lr] = v.z;
-        xs[(kq + 3) * kEstLd + lr] = v.w;
-        ws[(kq + 0) * ws_ld + lr] = u.x;
-        ws[(kq + 1) * ws_ld + lr] = u.y;
-        ws[(kq + 2) * ws_ld + lr] = u.z;
-        ws[(kq + 3) * ws_ld + lr] = u.w;
+      for (int q = 0; q < 4; ++q) store_split4(ahi, alo, xr, xc + q, xv[q]);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) store_split4(bhi, blo, tid, q, wv[q]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      ok = __syncthreads_and(ok);
+      if (!ok) break;
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t idesc = make_idesc_tf32(128, n1p);
+        const uint64_t dah = make_sdesc_sw128(smem_u32(ahi), 16, 1024), dal = make_sdesc_sw128(smem_u32(alo), 16, 1024);
+        const uint64_t dbh = make_sdesc_sw128(smem_u32(bhi), 16, 1024), dbl = make_sdesc_sw128(smem_u32(blo), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t off = (uint64_t)((kk * 32) >> 4);
+          umma_tf32_ss(tmem + kEstAcc1, dah + off, dbh + off, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+          umma_tf32_ss(tmem + kEstAcc1, dah + off, dbl + off, idesc, 1u);
+          umma_tf32_ss(tmem + kEstAcc1, dal + off, dbh + off, idesc, 1u);
+        }
+        umma_commit(smem_u32(&bars[use & 1]));
       }
-      __syncthreads();
-#pragma unroll 8
-      for (int kk = 0; kk < kEstK; ++kk) {
-        const float4 a = *reinterpret_cast<const float4*>(xs + kk * kEstLd + ty * 4);
-        const float4 b = *reinterpret_cast<const float4*>(ws + kk * ws_ld + tx * 4);
-        const float av[4] = {a.x, a.y, a.z, a.w};
-        const float bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-      }
+      ++use;
     }
+    if (!ok) break;
+    // every layer-1 product of this pass has completed
+    if (tid == 0) umma_commit(smem_u32(&bars[2]));
+    ok = mbar_wait(smem_u32(&bars[2]), done_phase & 1, abort, timeout_ns);
+    ++done_phase;
+    tc_fence_after();
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    // ------------------------------------------------------------ layer 2
+    for (int pi = 0; pi < (n1 + 31) / 32; ++pi) {
+      const int u0 = n0 + pi * 32;   // first hidden unit of this panel
+      ok = wait_stage(use) && ok;
+      uint8_t* st = stage(use);
+      uint8_t *ahi = st, *alo = st + kEstPanelA, *bhi = st + 2 * kEstPanelA, *blo = bhi + kEstPanelB;
+      if (warp < 4) {
+        // relu(acc1 + b1) for this thread's tile row and the panel's 32 units
+        const int r = warp * 32 + lane;
+        float v[32];
+        tmem_ld32(tmem + kEstAcc1 + ((uint32_t)(warp * 32) << 16) + (uint32_t)(pi * 32), v);
+        tmem_ld_wait();
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int unit = nb + tx * 4 + j;
-      if (unit < hidden) {
-        const float bias = B1[unit];
+        for (int c = 0; c < 8; ++c) {
+          float4 hv;
+          float* hp = reinterpret_cast<float*>(&hv);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) hs[unit * kEstLd + ty * 4 + i] = fmaxf(acc[i][j] + bias, 0.f);
+          for (int q = 0; q < 4; ++q) {
+            const int unit = u0 + c * 4 + q;
+            hp[q] = (unit < hidden) ? fmaxf(v[c * 4 + q] + __ldg(B1 + unit), 0.f) : 0.f;
+          }
+          store_split4(ahi, alo, r, c, hv);
+        }
+      } else {
+        // W2[o, u0 .. u0+31] for every output o
+        for (int t = tid - 128; t < E * 8; t += 128) {
+          const int o = t >> 3, c = t & 7;
+          const int unit = u0 + c * 4;
+          const float4 wv = (unit < hidden) ? __ldg(reinterpret_cast<const float4*>(W2 + (long long)o * hidden + unit))
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+          store_split4(bhi, blo, o, c, wv);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      ok = __syncthreads_and(ok);
+      if (!ok) break;
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t idesc = make_idesc_tf32(128, E);
+        const uint64_t dah = make_sdesc_sw128(smem_u32(ahi), 16, 1024), dal = make_sdesc_sw128(smem_u32(alo), 16, 1024);
+        const uint64_t dbh = make_sdesc_sw128(smem_u32(bhi), 16, 1024), dbl = make_sdesc_sw128(smem_u32(blo), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t off = (uint64_t)((kk * 32) >> 4);
+          umma_tf32_ss(tmem + kEstAcc2, dah + off, dbh + off, idesc, (acc2_started || kk > 0) ? 1u : 0u);
+          umma_tf32_ss(tmem + kEstAcc2, dah + off, dbl + off, idesc, 1u);
+          umma_tf32_ss(tmem + kEstAcc2, dal + off, dbh + off, idesc, 1u);
+        }
+        umma_commit(smem_u32(&bars[use & 1]));
+      }
+      acc2_started = true;
+      ++use;
+    }
+  }
+  // ------------------------------------------------------------ phi = acc2 + b2
+  if (ok) {
+    if (tid == 0) umma_commit(smem_u32(&bars[2]));
+    ok = mbar_wait(smem_u32(&bars[2]), done_phase & 1, abort, timeout_ns);
+    tc_fence_after();
+  }
+  ok = __syncthreads_and(ok);
+  if (ok && warp < 4) {
+    const int r = warp * 32 + lane;
+    float* out = phi + (((long long)which * G.B * G.heads + bh) * G.ntmax + j0 + r) * E;
+#pragma unroll
+    for (int c0 = 0; c0 < E; c0 += 32) {
+      float v[32];
+      tmem_ld32(tmem + kEstAcc2 + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+      tmem_ld_wait();
+      if (r < nrows) {
+#pragma unroll
+        for (int q = 0; q < 32 && c0 + q < E; q += 4) {
+          float4 o4 = make_float4(v[q] + __ldg(B2 + c0 + q), v[q + 1] + __ldg(B2 + c0 + q + 1),
+                                  v[q + 2] + __ldg(B2 + c0 + q + 2), v[q + 3] + __ldg(B2 + c0 + q + 3));
+          *reinterpret_cast<float4*>(out + c0 + q) = o4;
+        }
       }
     }
   }
-
-  // ---- layer 2: phi = hidden W2^T + b2
-  float acc2[4][CW];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int c = 0; c < CW; ++c) acc2[i][c] = 0.f;
-  for (int k0 = 0; k0 < hidden; k0 += kEstK) {
-    __syncthreads();
-    for (int t = tid; t < E * (kEstK / 4); t += 256) {
-      const int o = t % E, kq = (t / E) * 4;
-      float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (k0 + kq < hidden) u = *reinterpret_cast<const float4*>(W2 + (long long)o * hidden + k0 + kq);
-      ws[(kq + 0) * ws_ld + o] = u.x;
-      ws[(kq + 1) * ws_ld + o] = u.y;
-      ws[(kq + 2) * ws_ld + o] = u.z;
-      ws[(kq + 3) * ws_ld + o] = u.w;
-    }
-    __syncthreads();
-    const int kn = min(kEstK, hidden - k0);
-    for (int kk = 0; kk < kn; ++kk) {
-      const float4 a = *reinterpret_cast<const float4*>(hs + (k0 + kk) * kEstLd + ty * 4);
-      const float av[4] = {a.x, a.y, a.z, a.w};
-      float bv[CW];
-#pragma unroll
-      for (int c = 0; c < CW; ++c) bv[c] = ws[kk * ws_ld + tx * CW + c];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int c = 0; c < CW; ++c) acc2[i][c] = fmaf(av[i], bv[c], acc2[i][c]);
-    }
+  // Every MMA issued above completes before TMEM is released.
+  if (tid == 0) {
+    umma_commit(smem_u32(&bars[3]));
+    int dummy = 0;
+    mbar_wait(smem_u32(&bars[3]), 0, &dummy, timeout_ns);
   }
-  float* out = phi + (((long long)which * G.B * G.heads + bh) * G.ntmax + j0) * E;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = ty * 4 + i;
-    if (r < nrows) {
-#pragma unroll
-      for (int c = 0; c < CW; ++c) {
-        const int o = tx * CW + c;
-        out[(long long)r * E + o] = acc2[i][c] + B2[o];
-      }
-    }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kEstTmemCols);
   }
 }
 
-template <int CW>
+template <int E>
 static cudaError_t launch_est_t(const Geometry& G, const float* dq, const float* dk, const EstimatorWeights& wq,
-                                const EstimatorWeights& wk, int hidden, float* phi, cudaStream_t s) {
-  const size_t smem = estimator_smem_bytes(G.d, hidden, 16 * CW);
-  cudaError_t err = cudaFuncSetAttribute(estimator_kernel<CW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                                const EstimatorWeights& wk, int hidden, float* phi, uint64_t timeout_ns,
+                                cudaStream_t s) {
+  const size_t smem = estimator_smem_bytes(G.d, hidden, E);
+  cudaError_t err = cudaFuncSetAttribute(estimator_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid((G.ntmax + kEstRows - 1) / kEstRows, G.B * G.heads, 2);
-  estimator_kernel<CW><<<grid, 256, smem, s>>>(G, dq, dk, wq, wk, hidden, phi);
+  estimator_kernel<E><<<grid, kEstThreads, smem, s>>>(G, dq, dk, wq, wk, hidden, phi, timeout_ns);
   return cudaGetLastError();
 }
 
 cudaError_t launch_estimator(const Geometry& G, const float* dq, const float* dk, const EstimatorWeights& wq,
-                             const EstimatorWeights& wk, int hidden, int e, float* phi, cudaStream_t s) {
+                             const EstimatorWeights& wk, int hidden, int e, float* phi, uint64_t timeout_ns,
+                             cudaStream_t s) {
   switch (e) {
-    case 16: return launch_est_t<1>(G, dq, dk, wq, wk, hidden, phi, s);
-    case 32: return launch_est_t<2>(G, dq, dk, wq, wk, hidden, phi, s);
-    case 64: return launch_est_t<4>(G, dq, dk, wq, wk, hidden, phi, s);
-    case 128: return launch_est_t<8>(G, dq, dk, wq, wk, hidden, phi, s);
+    case 16: return launch_est_t<16>(G, dq, dk, wq, wk, hidden, phi, timeout_ns, s);
+    case 32: return launch_est_t<32>(G, dq, dk, wq, wk, hidden, phi, timeout_ns, s);
+    case 64: return launch_est_t<64>(G, dq, dk, wq, wk, hidden, phi, timeout_ns, s);
+    case 128: return launch_est_t<128>(G, dq, dk, wq, wk, hidden, phi, timeout_ns, s);
     default: return cudaErrorInvalidValue;
   }
 }

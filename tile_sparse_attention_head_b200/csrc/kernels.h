@@ -20,6 +20,7 @@ struct EstimatorWeights {
 struct TopkArgs {
   int32_t* idx;
   float* probs;
+  uint64_t timeout_ns;   // bounded-wait limit of the tensor-core estimator
   int32_t k_max;
   int32_t k_per_head[VEDA_MAX_HEADS];
 };
@@ -64,7 +65,8 @@ cudaError_t launch_tripool(const Geometry& G, const void* xp, float* desc, cudaS
 
 size_t estimator_smem_bytes(int d, int hidden, int e);
 cudaError_t launch_estimator(const Geometry& G, const float* dq, const float* dk, const EstimatorWeights& wq,
-                             const EstimatorWeights& wk, int hidden, int e, float* phi, cudaStream_t s);
+                             const EstimatorWeights& wk, int hidden, int e, float* phi, uint64_t timeout_ns,
+                             cudaStream_t s);
 void score_topk_config(int ntmax, int e, int* qb, int* ntpad, size_t* smem);
 cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const float* desc_k,
                               const EstimatorWeights& wq, const EstimatorWeights& wk, int hidden,

@@ -5,7 +5,8 @@
 //
 // Two kernels:
 //   estimator_kernel  phi = W2 relu(W1 desc + b1) + b2 for every Q and K tile,
-//                     fp32 on the CUDA cores, written to the workspace;
+//                     on the tensor cores at fp32 accuracy (estimator.cu),
+//                     written to the workspace;
 //   score_topk_kernel per block of Q-tile rows: s = phi_q phi_k^T / sqrt(e)
 //                     into shared memory, optional row softmax, then an exact
 //                     radix select of the k-th largest score per row and an
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(kScoreThreads)
 cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const float* desc_k,
                               const EstimatorWeights& wq, const EstimatorWeights& wk, int hidden,
                               int e, float* phi, const TopkArgs& args, cudaStream_t s) {
-  cudaError_t err = launch_estimator(G, desc_q, desc_k, wq, wk, hidden, e, phi, s);
+  cudaError_t err = launch_estimator(G, desc_q, desc_k, wq, wk, hidden, e, phi, args.timeout_ns, s);
   if (err != cudaSuccess) return err;
 
   int qb, ntpad;

@@ -324,6 +324,7 @@ veda_status veda_tile_score_topk(const veda_problem* p, const float* desc_q, con
   args.idx = idx;
   args.probs = probs;
   args.k_max = k_max;
+  args.timeout_ns = g_timeout_ns;
   EstimatorWeights wq{mlp_q->w1, mlp_q->b1, mlp_q->w2, mlp_q->b2};
   EstimatorWeights wk{mlp_k->w1, mlp_k->b1, mlp_k->w2, mlp_k->b2};
   cudaError_t ce = launch_score_topk(G, desc_q, desc_k, wq, wk, hidden, e, static_cast<float*>(workspace), args,
@@ -409,6 +410,7 @@ veda_status veda_tile_score_topk_noalloc(const veda_problem* p, const float* des
   args.idx = idx;
   args.probs = probs;
   args.k_max = k_max;
+  args.timeout_ns = g_timeout_ns;
   EstimatorWeights wq{mlp_q->w1, mlp_q->b1, mlp_q->w2, mlp_q->b2};
   EstimatorWeights wk{mlp_k->w1, mlp_k->b1, mlp_k->w2, mlp_k->b2};
   cudaError_t ce = launch_score_topk(G, desc_q, desc_k, wq, wk, hidden, e, scratch, args, (cudaStream_t)stream);
