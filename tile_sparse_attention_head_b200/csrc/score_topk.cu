@@ -26,10 +26,14 @@ __device__ __forceinline__ uint32_t float_key(float f) {
 }
 
 constexpr int kScoreThreads = 256;
-constexpr int kKChunk = 64;        // K tiles staged per step
+constexpr int kKChunk = 128;       // K tiles staged per step
+constexpr int kQRows = 16;         // most Q-tile rows per CTA (the score tile is 16 x 128)
 
-// grid: (ceil(NT_max / qb), B*heads).  Shared memory: scores [qb][ntmax_pad],
-// phi_q [qb][e], phi_k chunk [64][e+1], radix histograms [8][256].
+// grid: (ceil(NT_max / qb), B*heads), qb <= 16.  Shared memory: scores
+// [qb][ntmax_pad], phi_q^T [e][16], phi_k chunk^T [e][128] (both k-major, so
+// a score step is one float2 and one float4 load feeding 8 FMAs: thread t
+// forms rows 2(t/32), 2(t/32)+1 x columns 4(t%32)..+3 of the 16 x 128 tile),
+// radix histograms [8][256].
 __global__ void __launch_bounds__(kScoreThreads)
     score_topk_kernel(const __grid_constant__ Geometry G, const float* __restrict__ phi, int e,
                       int qb, int ntpad, const __grid_constant__ TopkArgs args) {
@@ -56,32 +60,56 @@ __global__ void __launch_bounds__(kScoreThreads)
   }
   const int nrows = min(qb, nt - i0);
   float* s_scores = sm;                            // [qb][ntpad]
-  float* s_phiq = s_scores + qb * ntpad;           // [qb][e]
-  float* s_phik = s_phiq + qb * e;                 // [64][e+1]
-  uint32_t* s_hist = reinterpret_cast<uint32_t*>(s_phik + kKChunk * (e + 1));  // [8][256]
+  float* s_phiq = s_scores + qb * ntpad;           // [e][16]
+  float* s_phik = s_phiq + e * kQRows;             // [e][128]
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(s_phik + e * kKChunk);  // [8][256]
 
   const float* phq = phi + ((long long)bh * G.ntmax + i0) * e;
   const float* phk = phi + (((long long)G.B * G.heads + bh) * G.ntmax) * e;
-  for (int i = tid; i < qb * e; i += kScoreThreads) s_phiq[i] = (i / e < nrows) ? phq[i] : 0.f;
+  for (int t = tid; t < kQRows * e; t += kScoreThreads) {
+    const int r = t % kQRows, cc = t / kQRows;
+    s_phiq[cc * kQRows + r] = (r < nrows) ? phq[(long long)r * e + cc] : 0.f;
+  }
   const float inv_sqrt_e = rsqrtf((float)e);
 
-  // Scores: thread -> column c = tid % 64 of the chunk, rows rg, rg+4, ...
-  const int c_local = tid % kKChunk, rg = tid / kKChunk;
+  // Scores, one 16 x 128 tile per chunk of K tiles.
+  const int cg = tid & 31, rp = tid >> 5;
   for (int jc = 0; jc < nt; jc += kKChunk) {
     __syncthreads();
     const int ncols = min(kKChunk, nt - jc);
-    for (int i = tid; i < kKChunk * e; i += kScoreThreads) {
-      const int jj = i / e, cc = i % e;
-      s_phik[jj * (e + 1) + cc] = (jj < ncols) ? phk[(long long)(jc + jj) * e + cc] : 0.f;
+    // phi_k rows jc .. jc+127, transposed; consecutive threads take
+    // consecutive rows, so the transposed stores do not conflict.
+    for (int t = tid; t < kKChunk * (e / 4); t += kScoreThreads) {
+      const int jj = t % kKChunk, q4 = t / kKChunk;
+      const float4 v = (jj < ncols) ? __ldg(reinterpret_cast<const float4*>(phk + (long long)(jc + jj) * e) + q4)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+      s_phik[(4 * q4 + 0) * kKChunk + jj] = v.x;
+      s_phik[(4 * q4 + 1) * kKChunk + jj] = v.y;
+      s_phik[(4 * q4 + 2) * kKChunk + jj] = v.z;
+      s_phik[(4 * q4 + 3) * kKChunk + jj] = v.w;
     }
     __syncthreads();
-    if (c_local < ncols) {
-      for (int r = rg; r < nrows; r += kScoreThreads / kKChunk) {
-        const float* a = s_phiq + r * e;
-        const float* b = s_phik + c_local * (e + 1);
-        float acc = 0.f;
-        for (int cc = 0; cc < e; ++cc) acc = fmaf(a[cc], b[cc], acc);
-        s_scores[r * ntpad + jc + c_local] = acc * inv_sqrt_e;
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll 8
+    for (int cc = 0; cc < e; ++cc) {
+      const float2 a = *reinterpret_cast<const float2*>(s_phiq + cc * kQRows + 2 * rp);
+      const float4 b = *reinterpret_cast<const float4*>(s_phik + cc * kKChunk + 4 * cg);
+      acc[0][0] = fmaf(a.x, b.x, acc[0][0]);
+      acc[0][1] = fmaf(a.x, b.y, acc[0][1]);
+      acc[0][2] = fmaf(a.x, b.z, acc[0][2]);
+      acc[0][3] = fmaf(a.x, b.w, acc[0][3]);
+      acc[1][0] = fmaf(a.y, b.x, acc[1][0]);
+      acc[1][1] = fmaf(a.y, b.y, acc[1][1]);
+      acc[1][2] = fmaf(a.y, b.z, acc[1][2]);
+      acc[1][3] = fmaf(a.y, b.w, acc[1][3]);
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int r = 2 * rp + q;
+      if (r < nrows) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (4 * cg + c < ncols) s_scores[r * ntpad + jc + 4 * cg + c] = acc[q][c] * inv_sqrt_e;
       }
     }
   }
@@ -207,12 +235,12 @@ cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const floa
 // Rows per CTA so that the score block fits in ~160 KB of shared memory.
 void score_topk_config(int ntmax, int e, int* qb, int* ntpad, size_t* smem) {
   const int pad = (ntmax + 3) & ~3;
-  int rows = (int)((160 * 1024) / (4 * (size_t)pad));
-  if (rows > 16) rows = 16;
+  int rows = (int)((140 * 1024) / (4 * (size_t)pad));
+  if (rows > kQRows) rows = kQRows;
   if (rows < 1) rows = 1;
   *qb = rows;
   *ntpad = pad;
-  *smem = sizeof(float) * ((size_t)rows * pad + (size_t)rows * e + (size_t)kKChunk * (e + 1)) +
+  *smem = sizeof(float) * ((size_t)rows * pad + (size_t)e * kQRows + (size_t)e * kKChunk) +
           sizeof(uint32_t) * 8 * 256;
 }
 
