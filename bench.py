@@ -155,11 +155,101 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of every rank's x (each rank's device-timed milliseconds)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(flops_per_rank: float, ms_max: float, world: int) -> float:
+    """Whole-job TFLOP/s: every rank runs its own layer, the job takes the slowest rank's time."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
+def tiles_per_head(w):
+    """Tiles of each head: the grid padded up to multiples of its tiling."""
+    return [(-(-w.T // pt)) * (-(-w.H // ph)) * (-(-w.W // pw)) for pt, ph, pw in w.tilings]
+
+
+def workload_for(args):
+    """The preset, with the keep ratio overridden by --keep or --fixed-k."""
+    import dataclasses
+    from veda_synth import PRESETS
+    w = PRESETS[args.workload]
+    if args.keep is not None:
+        w = dataclasses.replace(w, keep=float(args.keep))
+    if args.fixed_k is not None:
+        w = dataclasses.replace(w, keep=float(args.fixed_k) / max(tiles_per_head(w)))
+    return w
+
+
+def tile_token_counts(w):
+    """[heads, NT_max] number of token slots of every tile (0 past NT_h)."""
+    nts = tiles_per_head(w)
+    out = np.zeros((w.heads, max(nts)), dtype=np.int64)
+    for h, (pt, ph, pw) in enumerate(w.tilings):
+        nT, nH, nW = -(-w.T // pt), -(-w.H // ph), -(-w.W // pw)
+        j = np.arange(nts[h])
+        jt, jh, jw = j // (nH * nW), (j // nW) % nH, j % nW
+        out[h, :nts[h]] = (np.minimum(pt, w.T - jt * pt) * np.minimum(ph, w.H - jh * ph) *
+                           np.minimum(pw, w.W - jw * pw))
+    return out
+
+
+def useful_flops(w, idx):
+    """FLOPs of the kept (query, key) pairs that are both tokens (pad slots excluded)."""
+    cnt = tile_token_counts(w)                        # [heads, NT_max]
+    idx = idx.astype(np.int64)                        # [B, heads, NT_max, k_max]
+    sel = np.where(idx >= 0, idx, 0)
+    kv = np.take_along_axis(cnt[None, :, None, :].repeat(idx.shape[2], axis=2).repeat(idx.shape[0], axis=0),
+                            sel, axis=3)
+    kv = np.where(idx >= 0, kv, 0).sum(axis=3)        # valid keys per Q tile
+    return float((kv * cnt[None]).sum() * 4 * w.d)
+
+
+def tile_map_measure(V, w, p, qd, kd, args, rank):
+    """Times veda_tile_map_maxpool over a random 10% of Q tiles per head (the
+    distillation target), with its tensor and exponential bounds."""
+    from veda_synth import make_map_rows
+    dev = qd.device
+    ts = p.tile_shape()
+    qp = torch.empty(ts, dtype=torch.bfloat16, device=dev)
+    kp = torch.empty(ts, dtype=torch.bfloat16, device=dev)
+    V.veda_tile_permute(p, qd, qp)
+    V.veda_tile_permute(p, kd, kp)
+    rows = make_map_rows(p.nt_per_head, w.B, 0.1, seed=2)
+    R = rows.shape[1]
+    counts = (rows >= 0).sum(dim=1).view(w.B, w.heads).numpy()
+    rows = rows.to(dev)
+    ws = torch.empty(V.veda_tile_map_workspace(p, R) // 4 + 64, dtype=torch.float32, device=dev)
+    mp = torch.empty((w.B, w.heads, R, p.nt_max), dtype=torch.float32, device=dev)
+    for _ in range(2):
+        V.veda_tile_map_maxpool(p, qp, kp, rows, mp, ws)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.map_steps):
+        V.veda_tile_map_maxpool(p, qp, kp, rows, mp, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    V.veda_sync_status()
+    ms = e0.elapsed_time(e1) / args.map_steps
+    nts = np.asarray(p.nt_per_head)
+    keys = (counts * nts[None, :] * w.S).astype(np.float64)     # subset rows x all key slots
+    flops = float((2.0 * w.S * w.d * keys).sum())               # one Q K^T sweep
+    exps = float((w.S * keys).sum())
+    peaks, src = load_peaks()
+    tflops = flops / (ms * 1e-3) / 1e12
+    mufu_peak = 16 * 148 * peaks.get("sm_max_mhz", 1965.0) * 1e6   # ex2 per second at the maximum clock
+    return {"ms": ms, "subset_rows": int(counts.sum()), "flops": flops, "exps": exps, "tflops": tflops,
+            "roofline": {"bound": "tensor+exp", "achieved": tflops, "peak": peaks["bf16_tflops_sustained"],
+                         "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops_sustained"],
+                         "exp_rate": exps / (ms * 1e-3), "exp_peak_mufu": mufu_peak,
+                         "peak_source": f"{src} bf16 sustained; exp peak = 16 ex2/clk/SM at the maximum clock"}}
 
 
 def bench_config(w, args, world, flops):
@@ -205,7 +295,7 @@ def run_ours(args, world, rank, local):
     import tile_sparse_attention_head_b200 as V
     from veda_synth import PRESETS, make_mlp, make_qkv
 
-    w = PRESETS[args.workload]
+    w = workload_for(args)
     p = V.Problem(w.B, w.heads, w.d, w.S, (w.T, w.H, w.W), w.tilings)
     q, k, v = make_qkv(w, seed=rank)
     m = make_mlp(w, seed=1)
@@ -320,15 +410,20 @@ def run_ours(args, world, rank, local):
     sustained = None
     if args.attn_sustain > 0:
         sustained = attention_sustained(V, p, att, qd, kd, vd, out, args, flops, local)
-    res = {"metric": METRIC, "value": world * flops / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+    useful = useful_flops(w, att.idx.cpu().numpy())
+    tmap = tile_map_measure(V, w, p, qd, kd, args, rank) if args.map else None
+    res = {"metric": METRIC, "value": weak_scaling_value(flops, ms_step, world), "unit": "TFLOP/s",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
            "config": bench_config(w, args, world, flops),
            "ms_per_layer": ms_step, "stage_ms": stage_ms, "attn_tflops": achieved,
+           "useful_flops_per_layer": useful, "attn_useful_tflops": useful / (attn_ms * 1e-3) / 1e12,
            "pct_of_bf16_peak": 100.0 * achieved / peaks["bf16_tflops"],
            "roofline": roofline, "gpu_launches": launches_per_step * args.steps, "clocks": clk, "e2e": e2e}
     if sustained is not None:
         res["attention_sustained"] = sustained
+    if tmap is not None:
+        res["tile_map"] = tmap
     return res, (w, p, ks, flops)
 
 
@@ -364,9 +459,8 @@ def cpu_sample_oracle(w, p_nts, ks, heads=1, tiles=None, seed=0):
 
 def run_reference(args, world, rank):
     """The fp64 CPU oracle as the reference arm, timed on the host cores."""
-    from veda_synth import PRESETS
     from oracle import veda_oracle as O
-    w = PRESETS[args.workload]
+    w = workload_for(args)
     nts, _ = O.tile_layout((w.T, w.H, w.W), w.tilings)
     ks = [O.keep_count(n, float(np.float32(w.keep))) for n in nts]
     tiles = args.ref_tiles
@@ -399,6 +493,11 @@ def main():
     ap.add_argument("--layout", choices=["tile", "grid"], default="grid",
                     help="tile-major copies (permute/unpermute steps) or grid order throughout")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--keep", type=float, default=None, help="override the preset's keep ratio")
+    ap.add_argument("--fixed-k", type=int, default=None,
+                    help="keep ratio k / NT_max, i.e. k selected tiles per Q tile (the fixed-k token sweep)")
+    ap.add_argument("--map", action="store_true", help="also time the max-pooled tile map (10%% of Q tiles)")
+    ap.add_argument("--map-steps", type=int, default=5)
     ap.add_argument("--attn-sustain", type=float, default=0.0,
                     help="also run the attention kernel back to back for this many seconds, sampling clock and power")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -1,0 +1,80 @@
+"""Host-side logic of bench.py, on the CPU: tile token counts, useful FLOPs,
+the fixed-k sweep override, and the multi-rank timing reduction on two gloo
+ranks (the path bench.py takes under torchrun, minus the GPUs)."""
+import argparse
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from oracle import veda_oracle as O  # noqa: E402
+from veda_synth import PRESETS  # noqa: E402
+
+from parity import SMALL  # noqa: E402
+
+
+@pytest.mark.parametrize("w", SMALL + [PRESETS["wan14b"]], ids=[w.name for w in SMALL] + ["wan14b"])
+def test_tile_token_counts_match_the_oracle_layout(w):
+    cnt = bench.tile_token_counts(w)
+    nts, ntmax = O.tile_layout((w.T, w.H, w.W), w.tilings)
+    assert cnt.shape == (w.heads, ntmax)
+    assert bench.tiles_per_head(w) == list(nts)
+    for h in range(w.heads):
+        tab = O.slot_table((w.T, w.H, w.W), w.tilings[h])
+        ref = (tab.reshape(nts[h], w.S) >= 0).sum(axis=1)
+        np.testing.assert_array_equal(cnt[h, :nts[h]], ref)
+        assert np.all(cnt[h, nts[h]:] == 0)
+
+
+def test_useful_flops_of_a_dense_selection_is_n_squared():
+    w = SMALL[1]
+    nts, ntmax = O.tile_layout((w.T, w.H, w.W), w.tilings)
+    idx = np.full((w.B, w.heads, ntmax, ntmax), -1, dtype=np.int32)
+    for h in range(w.heads):
+        idx[:, h, :nts[h], :nts[h]] = np.arange(nts[h])
+    N = w.T * w.H * w.W
+    assert bench.useful_flops(w, idx) == pytest.approx(w.B * w.heads * N * N * 4 * w.d)
+    # with -1 padding and invalid Q rows nothing is counted
+    idx[:, :, :, 1:] = -1
+    cnt = bench.tile_token_counts(w)
+    expect = sum(int((cnt[h, :nts[h]] * cnt[h, 0]).sum()) for h in range(w.heads)) * w.B * 4 * w.d
+    assert bench.useful_flops(w, idx) == pytest.approx(expect)
+
+
+@pytest.mark.parametrize("name", ["sweep61k", "sweep123k", "sweep246k"])
+def test_fixed_k_override_keeps_k_tiles(name):
+    args = argparse.Namespace(workload=name, keep=None, fixed_k=26)
+    w = bench.workload_for(args)
+    nts, _ = O.tile_layout((w.T, w.H, w.W), w.tilings)
+    assert {O.keep_count(n, float(np.float32(w.keep))) for n in nts} == {26}
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.barrier(world)
+        ms = bench.max_over_ranks(10.0 + 5.0 * rank, world)
+        out[rank] = ms
+        bench.barrier(world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_on_two_gloo_ranks():
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    out = mp.get_context("spawn").Manager().dict()
+    mp.spawn(_rank_main, args=(2, port, out), nprocs=2, join=True)
+    assert dict(out) == {0: 15.0, 1: 15.0}
+    assert bench.weak_scaling_value(7.8e12, 15.0, 2) == pytest.approx(2 * 7.8e12 / 15e-3 / 1e12)
