@@ -158,3 +158,33 @@ def test_grid_wan14b_full_size_sampled(V):
     V.veda_sync_status()
     assert torch.equal(idx_g, att_t.idx)
     assert torch.equal(out_g, out_t)
+
+
+def test_extreme_score_in_the_last_key_slot(V):
+    """One key, in the last slot of a tile, scores about 300 (log2 units) above every
+    other key of a query row: the exponent reference must take it into account, or
+    the exponentials of that row overflow."""
+    from parity import wl
+    w = wl("extreme", (4, 16, 16), 1, 1, 128, 128, [(2, 8, 8)], 1.0, 256, 64)
+    p = _problem(V, w)
+    q, k, v = make_qkv(w, seed=7)
+    grid = (w.T, w.H, w.W)
+    pt, ph, pw = w.tilings[0]
+    n_last = ((pt - 1) * w.H + (ph - 1)) * w.W + (pw - 1)     # slot S-1 of tile 0
+    qrow = q[0, 0, 0].float()
+    k[0, 0, n_last] = (qrow * (2400.0 / float(qrow @ qrow))).to(torch.bfloat16)
+    nt = p.nt_per_head[0]
+    idx = torch.arange(nt, dtype=torch.int32).expand(w.B, w.heads, p.nt_max, nt).contiguous()
+    o = torch.empty(p.grid_shape(), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((p.B, p.heads, p.N), dtype=torch.float32, device="cuda")
+    V.veda_tile_sparse_attn_grid(p, q.cuda(), k.cuda(), v.cuda(), idx.cuda(), o, lse)
+    V.veda_sync_status()
+    qp, kp, vp = (O.tile_permute(f64(t), grid, w.tilings, w.S) for t in (q, k, v))
+    ref_op, ref_lse = O.sparse_attention(qp, kp, vp, idx.numpy(), grid, w.tilings, w.S)
+    ref_o = O.tile_unpermute(ref_op, grid, w.tilings, w.S)
+    ref_l = O.tile_unpermute(ref_lse[..., None], grid, w.tilings, w.S)[..., 0]
+    g, gl = f64(o), f64(lse)
+    assert np.all(np.isfinite(g)) and np.all(np.isfinite(gl))
+    assert ref_l[0, 0, 0] > 150.0                               # the extreme row really is extreme
+    check_attn_rows(g[0, 0], ref_o[0, 0])
+    assert np.abs(gl[0, 0] - ref_l[0, 0]).max() <= LSE_ABS

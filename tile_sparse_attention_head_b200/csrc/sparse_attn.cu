@@ -424,7 +424,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int c = 8; c + 16 <= BN; c += 16)
 #pragma unroll
         for (int q = 0; q < 8; ++q) m8[q] = fmax3(m8[q], sc[c + q], sc[c + 8 + q]);
-      if constexpr (BN % 16 == 8) {
+      if constexpr ((BN - 8) % 16 == 8) {   // the last 8 columns
 #pragma unroll
         for (int q = 0; q < 8; ++q) m8[q] = fmaxf(m8[q], sc[BN - 8 + q]);
       }

@@ -10,9 +10,12 @@
 // where rowmax_j(q) is the largest scaled logit (log2 units) of row q over
 // tile j and lse2(q) the row's log2-sum-exp2.  So:
 //   pass 1 (tcgen05): one CTA per subset Q tile streams every K tile of the
-//           head through the tensor cores (S = Q K^T in TMEM), and the
-//           softmax warps record rowmax_j(q) for every (q, j) in the
-//           workspace while accumulating the online log-sum-exp;
+//           head through the tensor cores (S = Q K^T into one of two TMEM
+//           buffers), and two softmax streams -- even and odd K tiles, one
+//           S buffer each, so two softmax warps share every scheduler --
+//           record rowmax_j(q) for every (q, j) in the workspace while
+//           accumulating an online log-sum-exp; the two partial sums are
+//           merged exactly at the end;
 //   pass 2: a warp per (Q tile, K tile) reads the 128 recorded maxima and
 //           the row lse2 values and takes the max of 2^(rowmax - lse2) over
 //           the token rows of the Q tile.
@@ -24,15 +27,15 @@
 
 namespace veda {
 
-// Pass 1 is exponential-bound (Q K^T only); one exponential in
-// kMapPolyEvery runs on the FMA pipe (exp2_fma), the rest on the
-// special-function unit.
-constexpr int kMapPolyEvery = 3;
+// Pass 1 is exponential-bound (Q K^T only): three pairs of exponentials in
+// eight run on the FMA pipe (exp2_fma_x2), the rest on the special-function
+// unit.
+__host__ __device__ constexpr bool map_poly_pair(int pair) { return (pair * 3) % 8 < 3; }
 
 template <int D, int BN>
 struct MapCfg {
   static constexpr int BM = 128;
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 320;   // producer, MMA issuer, two softmax warpgroups
   static constexpr int kStages = 4;
   static constexpr int kChunk = 128 * 128;
   static constexpr int kQBytes = BM * D * 2;
@@ -41,8 +44,9 @@ struct MapCfg {
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffBar = kOffK + kStages * kKBytes;
   static constexpr int kOffMisc = kOffBar + 16 * 8;
+  static constexpr int kOffRed = kOffMisc + 64;   // float [2: m, l][128 rows] of stream B
   static constexpr uint32_t kTmemCols = 256;
-  static constexpr size_t kSmem = 1024 + kOffMisc + 64;
+  static constexpr size_t kSmem = 1024 + kOffRed + 2 * 128 * 4;
 };
 
 enum {
@@ -51,7 +55,8 @@ enum {
   MBAR_KEMPTY = 5,  // +stage (4)
   MBAR_SFULL = 9,   // +buffer (2)
   MBAR_SFREE = 11,  // +buffer (2)
-  MBAR_DRAIN = 13
+  MBAR_DRAIN = 13,
+  MBAR_XFIN = 14    // stream B's final (m, l) are in shared memory (128 arrivals)
 };
 
 __device__ __forceinline__ bool map_warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
@@ -61,7 +66,7 @@ __device__ __forceinline__ bool map_warp_wait(uint32_t bar, uint32_t parity, vol
 }
 
 template <int D, int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     tile_map_pass1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ Geometry G, const __grid_constant__ MapArgs A) {
   using C = MapCfg<D, BN>;
@@ -96,6 +101,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(bar(MBAR_SFREE + s), 4);
     }
     mbar_init(bar(MBAR_DRAIN), 1);
+    mbar_init(bar(MBAR_XFIN), 128);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -173,66 +179,111 @@ __global__ void __launch_bounds__(192, 1)
     int dummy = 0;
     mbar_wait(bar(MBAR_DRAIN), 0, &dummy, tmo);
   } else {
-    const int quarter = warp & 3;
+    // ------------------------------------------------------------ softmax streams
+    const int sb = (warp - 2) >> 2;        // stream: K tiles t with t % 2 == sb, S buffer sb
+    const int quarter = warp & 3;          // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
-    const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(sb * 128);
     const float sl2 = A.scale_log2;
+    const uint64_t scl2 = f2(sl2, sl2);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     float* rm = A.rowmax + (((long long)bh * A.R + r) * G.ntmax) * S + row;
-    for (int t = 0; t < nt; ++t) {
-      const int sb = t & 1;
-      if (!(ok = map_warp_wait(bar(MBAR_SFULL + sb), (t >> 1) & 1, abort, tmo))) break;
-      tc_fence_after();
-      float s[BN];
+    // Slot offsets (t, y, x) of this lane's key columns c = 32 w + lane.
+    int8_t kt[BN / 32], ky[BN / 32], kx[BN / 32];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_lane + sb * 128 + c * 32, &s[c * 32]);
+    for (int w = 0; w < BN / 32; ++w) {
+      const int c = w * 32 + lane;
+      kx[w] = (int8_t)(c % hg.pw);
+      ky[w] = (int8_t)((c / hg.pw) % hg.ph);
+      kt[w] = (int8_t)(c / (hg.pw * hg.ph));
+    }
+    // Tile coordinates of t = sb, advanced by 2 tiles per step without division.
+    int jw = sb % hg.nTw, jh = (sb / hg.nTw) % hg.nTh, jt = sb / (hg.nTw * hg.nTh);
+    for (int t = sb; t < nt; t += 2) {
+      const int k = t >> 1;
+      if (!(ok = map_warp_wait(bar(MBAR_SFULL + sb), k & 1, abort, tmo))) break;
+      tc_fence_after();
+      float sc[BN];
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(t_lane + c * 32, &sc[c * 32]);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(MBAR_SFREE + sb));
 
-      const int jw = t % hg.nTw, jh = (t / hg.nTw) % hg.nTh, jt = t / (hg.nTw * hg.nTh);
       const int ct = min((int)hg.pt, G.T - jt * hg.pt);
       const int ch = min((int)hg.ph, G.H - jh * hg.ph);
       const int cw = min((int)hg.pw, G.W - jw * hg.pw);
       if (ct * ch * cw != S) {
         uint32_t mw[BN / 32];
 #pragma unroll
-        for (int w = 0; w < BN / 32; ++w) {
-          const int c = w * 32 + lane;
-          const int lw = c % hg.pw, lh = (c / hg.pw) % hg.ph, lt = c / (hg.pw * hg.ph);
-          mw[w] = __ballot_sync(0xffffffffu, lt < ct && lh < ch && lw < cw);
-        }
+        for (int w = 0; w < BN / 32; ++w) mw[w] = __ballot_sync(0xffffffffu, kt[w] < ct && ky[w] < ch && kx[w] < cw);
 #pragma unroll
         for (int c = 0; c < BN; ++c)
-          if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
+          if (!((mw[c >> 5] >> (c & 31)) & 1u)) sc[c] = -INFINITY;
       }
+      jw += 2;
+      while (jw >= hg.nTw) {
+        jw -= hg.nTw;
+        if (++jh == hg.nTh) {
+          jh = 0;
+          ++jt;
+        }
+      }
+      // Row maximum of the tile: three-input max over 8 chains.
       float m8[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) m8[q] = s[q];
+      for (int q = 0; q < 8; ++q) m8[q] = sc[q];
 #pragma unroll
-      for (int c = 8; c < BN; c += 8)
+      for (int c = 8; c + 16 <= BN; c += 16)
 #pragma unroll
-        for (int q = 0; q < 8; ++q) m8[q] = fmaxf(m8[q], s[c + q]);
-      float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      mt *= sl2;
+        for (int q = 0; q < 8; ++q) m8[q] = fmax3(m8[q], sc[c + q], sc[c + 8 + q]);
+      if constexpr ((BN - 8) % 16 == 8) {   // the last 8 columns
+#pragma unroll
+        for (int q = 0; q < 8; ++q) m8[q] = fmaxf(m8[q], sc[BN - 8 + q]);
+      }
+      const float mt = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * sl2;
       if (row < S) rm[(long long)t * S] = mt;
       const float m_new = fmaxf(m_run, mt);
-      float r8[8];
+      const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
+      const uint64_t nref2 = f2(-m_ref, -m_ref);
+      uint64_t r4[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int q = 0; q < 8; ++q) r8[q] = 0.f;
-#pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        const float x = fmaf(s[c], sl2, -m_new);
-        r8[c & 7] += (c % kMapPolyEvery == kMapPolyEvery - 1) ? exp2_fma(x) : fast_exp2(x);
+      for (int c = 0; c < BN; c += 2) {
+        float x0, x1, p0, p1;
+        f2_split(f2_fma(f2(sc[c], sc[c + 1]), scl2, nref2), x0, x1);
+        if (map_poly_pair(c >> 1)) {
+          exp2_fma_x2(x0, x1, p0, p1);
+        } else {
+          p0 = fast_exp2(x0);
+          p1 = fast_exp2(x1);
+        }
+        r4[(c >> 1) & 3] = f2_add(r4[(c >> 1) & 3], f2(p0, p1));
       }
-      const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
-      l_run = l_run * fast_exp2(m_run - m_new) + rs;
+      float ra, rb, rc, rd;
+      f2_split(f2_add(r4[0], r4[1]), ra, rb);
+      f2_split(f2_add(r4[2], r4[3]), rc, rd);
+      const float rs = (ra + rb) + (rc + rd);
+      l_run = (m_run == -INFINITY ? 0.f : l_run * fast_exp2(m_run - m_ref)) + rs;
       m_run = m_new;
     }
-    if (ok && row < S) A.lse2[((long long)bh * A.R + r) * S + row] = m_run + log2f(l_run);
+    // Merge the streams: stream B hands its (m, l) to stream A.
+    float* red = reinterpret_cast<float*>(smem + C::kOffRed);
+    if (sb == 1) {
+      red[row] = m_run;
+      red[128 + row] = l_run;
+      mbar_arrive(bar(MBAR_XFIN));
+    } else {
+      if (ok) ok = map_warp_wait(bar(MBAR_XFIN), 0, abort, tmo);
+      if (ok && row < S) {
+        const float mB = red[row], lB = red[128 + row];
+        const float m = fmaxf(m_run, mB);
+        const float l = (m_run == -INFINITY ? 0.f : l_run * fast_exp2(m_run - m)) +
+                        (mB == -INFINITY ? 0.f : lB * fast_exp2(mB - m));
+        A.lse2[((long long)bh * A.R + r) * S + row] = m + log2f(l);
+      }
+    }
   }
 
   tc_fence_before();
