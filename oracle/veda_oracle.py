@@ -330,3 +330,85 @@ def forward(q, k, v, grid, tilings, S, mlp_q, mlp_k, keep_ratio, scale=None):
     o = tile_unpermute(op, grid, tilings, S)
     return dict(qp=qp, kp=kp, vp=vp, desc_q=dq, desc_k=dk, idx=idx, probs=probs, scores=scores,
                 op=op, lse=lse, o=o)
+
+
+# --------------------------------------------------------------------------
+# Training the estimator -- row-wise KL distillation (section 2.1,
+# "Optimization": the predicted distribution of tile scores is aligned with
+# the full-attention reference row by row with a KL divergence; gradients do
+# not flow into the backbone features that feed the estimator).
+# --------------------------------------------------------------------------
+def distill_row_loss(m_row: np.ndarray, s_row: np.ndarray) -> float:
+    """KL(T || P) for one row, over the entries given (the head's valid K tiles):
+    T = m_row / sum(m_row), the max-pooled full-attention row as a distribution;
+    P = softmax(s_row), the estimator's row distribution.  Terms with T = 0
+    contribute 0."""
+    t = np.asarray(m_row, np.float64) / float(np.sum(m_row))
+    s = np.asarray(s_row, np.float64)
+    log_p = s - s.max() - math.log(float(np.exp(s - s.max()).sum()))
+    nz = t > 0
+    return float(np.sum(t[nz] * (np.log(t[nz]) - log_p[nz])))
+
+
+def _estimator_with_hidden(desc, w1, b1, w2, b2):
+    """Forward pass of estimator_head keeping the pre-activation z and the hidden a."""
+    z = desc @ np.asarray(w1, np.float64).T + np.asarray(b1, np.float64)
+    a = np.maximum(z, 0.0)
+    return z, a, a @ np.asarray(w2, np.float64).T + np.asarray(b2, np.float64)
+
+
+def distill_loss_grads(desc_q, desc_k, grid, tilings, S, mlp_q, mlp_k, tile_map, rows):
+    """L = mean over the subset rows (b, h, r) with rows[b*heads+h, r] >= 0 of
+    KL(T || P), with T the map row tile_map[b, h, r, :NT_h] normalised to sum 1
+    and P = softmax_j s[i, j] over j < NT_h, i = rows[b*heads+h, r]
+    (s = <phi_q(i), phi_k(j)> / sqrt(e) as in tile_scores_head).
+
+    Returns (L, grads_q, grads_k); each grads tuple matches (W1, b1, W2, b2)
+    of its estimator.  The descriptors are inputs only (the stop-gradient on
+    the backbone features).  Reading: the direction KL(target || predicted)
+    and the mean over rows are the plainest reading of "row-wise KL
+    distillation objective"; the derivative of ReLU at 0 is taken as 0.
+    """
+    desc_q = np.asarray(desc_q, np.float64)
+    desc_k = np.asarray(desc_k, np.float64)
+    tile_map = np.asarray(tile_map, np.float64)
+    rows = np.asarray(rows)
+    B, heads = desc_q.shape[:2]
+    nts, _ = tile_layout(grid, tilings)
+    valid = [(b, h, r) for b in range(B) for h in range(heads) for r in range(rows.shape[1])
+             if 0 <= rows[b * heads + h, r] < nts[h]]
+    n_rows = len(valid)
+    gq = [np.zeros(np.shape(w), np.float64) for w in mlp_q]
+    gk = [np.zeros(np.shape(w), np.float64) for w in mlp_k]
+    loss = 0.0
+    for b in range(B):
+        for h in range(heads):
+            nt = nts[h]
+            wq = tuple(np.asarray(w, np.float64)[h] for w in mlp_q)
+            wk = tuple(np.asarray(w, np.float64)[h] for w in mlp_k)
+            zq, aq, phq = _estimator_with_hidden(desc_q[b, h, :nt], *wq)
+            zk, ak, phk = _estimator_with_hidden(desc_k[b, h, :nt], *wk)
+            e = phq.shape[1]
+            dphq = np.zeros_like(phq)
+            dphk = np.zeros_like(phk)
+            for r in range(rows.shape[1]):
+                i = int(rows[b * heads + h, r])
+                if not 0 <= i < nt:
+                    continue
+                s = phq[i] @ phk.T / math.sqrt(e)
+                m = tile_map[b, h, r, :nt]
+                loss += distill_row_loss(m, s)
+                p = np.exp(s - s.max())
+                p /= p.sum()
+                g = (p - m / m.sum()) / n_rows          # dL/ds[i, :]
+                dphq[i] += g @ phk / math.sqrt(e)
+                dphk += np.outer(g, phq[i]) / math.sqrt(e)
+            # back through phi = W2 a + b2, a = relu(z), z = W1 desc + b1
+            for dph, z, a, desc, w, grad in ((dphq, zq, aq, desc_q[b, h, :nt], wq, gq),
+                                             (dphk, zk, ak, desc_k[b, h, :nt], wk, gk)):
+                grad[2][h] += dph.T @ a
+                grad[3][h] += dph.sum(axis=0)
+                dz = (dph @ w[2]) * (z > 0)
+                grad[0][h] += dz.T @ desc
+                grad[1][h] += dz.sum(axis=0)
+    return loss / max(n_rows, 1), tuple(gq), tuple(gk)

@@ -358,3 +358,89 @@ def test_forward_tiny_shapes_and_full_keep_reduction():
     out = O.forward(q, k, v, grid, w.tilings, w.S, mlp, mlp, w.keep)
     assert out["idx"].shape == (1, 2, 4, 2)
     assert np.all(out["idx"] >= 0)
+
+
+# ---------------------------------------------------------------- distillation loss and gradients
+def _distill_case(seed=0, B=1, heads=2, d=8, hidden=12, e=4, grid=(3, 4, 6), tilings=((1, 2, 4), (2, 2, 2)), S=8):
+    rng = np.random.default_rng(seed)
+    nts, ntmax = O.tile_layout(grid, tilings)
+    dq = rng.standard_normal((B, heads, ntmax, 3 * d))
+    dk = rng.standard_normal((B, heads, ntmax, 3 * d))
+    mk = lambda: (rng.standard_normal((heads, hidden, 3 * d)) * 0.4, rng.standard_normal((heads, hidden)) * 0.2,
+                  rng.standard_normal((heads, e, hidden)) * 0.4, rng.standard_normal((heads, e)) * 0.2)
+    mlp_q, mlp_k = mk(), mk()
+    R = 3
+    rows = np.full((B * heads, R), -1, dtype=np.int64)
+    for bh in range(B * heads):
+        h = bh % heads
+        rows[bh, : min(R, nts[h])] = rng.choice(nts[h], size=min(R, nts[h]), replace=False)
+    rows[0, -1] = -1                                   # an unused subset slot
+    tmap = np.zeros((B, heads, R, ntmax))
+    for b in range(B):
+        for h in range(heads):
+            tmap[b, h, :, :nts[h]] = rng.uniform(0.01, 1.0, (R, nts[h]))
+    return dict(desc_q=dq, desc_k=dk, grid=grid, tilings=tilings, S=S, mlp_q=mlp_q, mlp_k=mlp_k,
+                tile_map=tmap, rows=rows)
+
+
+def test_distill_row_loss_matches_scipy_kl():
+    from scipy.special import softmax
+    from scipy.stats import entropy
+    rng = np.random.default_rng(4)
+    for n in (1, 5, 37):
+        m = rng.uniform(0.0, 1.0, n)
+        m[0] = max(m[0], 1e-3)
+        if n > 2:
+            m[1] = 0.0                                  # a zero target entry
+        s = rng.standard_normal(n) * 3
+        assert O.distill_row_loss(m, s) == pytest.approx(entropy(m / m.sum(), softmax(s)), rel=1e-12, abs=1e-14)
+
+
+def test_distill_gradients_match_central_differences():
+    c = _distill_case()
+    loss, gq, gk = O.distill_loss_grads(**c)
+    assert loss > 0
+    rng = np.random.default_rng(7)
+    h = 1e-6
+    for side, grads in (("mlp_q", gq), ("mlp_k", gk)):
+        for t in range(4):
+            w = c[side][t]
+            for _ in range(6):
+                pos = tuple(rng.integers(0, s) for s in w.shape)
+                old = w[pos]
+                w[pos] = old + h
+                lp = O.distill_loss_grads(**c)[0]
+                w[pos] = old - h
+                lm = O.distill_loss_grads(**c)[0]
+                w[pos] = old
+                fd = (lp - lm) / (2 * h)
+                assert grads[t][pos] == pytest.approx(fd, rel=1e-5, abs=1e-9), (side, t, pos)
+
+
+def test_distill_gradient_of_the_k_side_output_bias_vanishes():
+    """A shift of phi_k's bias adds the same amount to every score of a row, which a
+    row softmax ignores, so dL/db2 of the K side is zero."""
+    c = _distill_case(seed=3)
+    _, gq, gk = O.distill_loss_grads(**c)
+    scale = max(np.abs(g).max() for g in gk[:3])
+    assert np.abs(gk[3]).max() <= 1e-12 * max(scale, 1.0)
+    assert np.abs(gq[3]).max() > 1e-6                  # the Q side's is not
+
+
+def test_distill_loss_and_gradients_vanish_when_the_target_is_the_prediction():
+    c = _distill_case(seed=5)
+    nts, _ = O.tile_layout(c["grid"], c["tilings"])
+    B, heads = c["desc_q"].shape[:2]
+    for b in range(B):
+        for h in range(heads):
+            wq = tuple(w[h] for w in c["mlp_q"])
+            wk = tuple(w[h] for w in c["mlp_k"])
+            s = O.tile_scores_head(c["desc_q"][b, h, :nts[h]], c["desc_k"][b, h, :nts[h]], wq, wk)
+            for r in range(c["rows"].shape[1]):
+                i = c["rows"][b * heads + h, r]
+                if i >= 0:
+                    c["tile_map"][b, h, r, :nts[h]] = 3.0 * O.row_softmax(s[i:i + 1])[0]   # any positive scale
+    loss, gq, gk = O.distill_loss_grads(**c)
+    assert abs(loss) < 1e-13
+    for g in gq + gk:
+        assert np.abs(g).max() < 1e-12
