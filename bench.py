@@ -210,7 +210,7 @@ def useful_flops(w, idx):
     return float((kv * cnt[None]).sum() * 4 * w.d)
 
 
-def tile_map_measure(V, w, p, qd, kd, args, rank):
+def tile_map_measure(V, w, p, qd, kd, args, rank, att=None):
     """Times veda_tile_map_maxpool over a random 10% of Q tiles per head (the
     distillation target), with its tensor and exponential bounds."""
     from veda_synth import make_map_rows
@@ -238,6 +238,28 @@ def tile_map_measure(V, w, p, qd, kd, args, rank):
     torch.cuda.synchronize()
     V.veda_sync_status()
     ms = e0.elapsed_time(e1) / args.map_steps
+    # the estimator's distillation step against this map (forward estimator,
+    # row-wise KL, gradients of both MLPs)
+    dist = None
+    if att is not None:
+        wt = (att._wq, att._wk)
+        grads = [tuple(torch.empty_like(t) for t in ws_) for ws_ in wt]
+        gq, gk = V.make_mlp_grad(*grads[0]), V.make_mlp_grad(*grads[1])
+        loss = torch.empty(1, dtype=torch.float32, device=dev)
+        dws = torch.empty(V.veda_distill_workspace(p, att.mlp_q.hidden, att.mlp_q.e, R) // 4 + 64,
+                          dtype=torch.float32, device=dev)
+        step = lambda: V.veda_distill_loss_grad(p, att.desc_q, att.desc_k, att.mlp_q, att.mlp_k, mp, rows, loss,
+                                                gq, gk, dws)
+        for _ in range(2):
+            step()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(args.map_steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+        V.veda_sync_status()
+        dist = {"ms": e0.elapsed_time(e1) / args.map_steps, "loss": float(loss.item())}
     nts = np.asarray(p.nt_per_head)
     keys = (counts * nts[None, :] * w.S).astype(np.float64)     # subset rows x all key slots
     flops = float((2.0 * w.S * w.d * keys).sum())               # one Q K^T sweep
@@ -246,6 +268,7 @@ def tile_map_measure(V, w, p, qd, kd, args, rank):
     tflops = flops / (ms * 1e-3) / 1e12
     mufu_peak = 16 * 148 * peaks.get("sm_max_mhz", 1965.0) * 1e6   # ex2 per second at the maximum clock
     return {"ms": ms, "subset_rows": int(counts.sum()), "flops": flops, "exps": exps, "tflops": tflops,
+            "distill_step": dist,
             "roofline": {"bound": "tensor+exp", "achieved": tflops, "peak": peaks["bf16_tflops_sustained"],
                          "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops_sustained"],
                          "exp_rate": exps / (ms * 1e-3), "exp_peak_mufu": mufu_peak,
@@ -411,7 +434,7 @@ def run_ours(args, world, rank, local):
     if args.attn_sustain > 0:
         sustained = attention_sustained(V, p, att, qd, kd, vd, out, args, flops, local)
     useful = useful_flops(w, att.idx.cpu().numpy())
-    tmap = tile_map_measure(V, w, p, qd, kd, args, rank) if args.map else None
+    tmap = tile_map_measure(V, w, p, qd, kd, args, rank, att) if args.map else None
     res = {"metric": METRIC, "value": weak_scaling_value(flops, ms_step, world), "unit": "TFLOP/s",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",

@@ -88,6 +88,16 @@ typedef struct {
   int32_t hidden, e;
 } veda_mlp;
 
+/* Gradient outputs for one estimator, DEVICE fp32, shaped like its weights:
+ * w1 [heads, hidden, 3d], b1 [heads, hidden], w2 [heads, e, hidden],
+ * b2 [heads, e]; 16-byte aligned; written in full by the call. */
+typedef struct {
+  float* w1;
+  float* b1;
+  float* w2;
+  float* b2;
+} veda_mlp_grad;
+
 /* ---------------------------------------------------------------- host helpers */
 
 /* Tiles per head after padding, NT_h = ceil(T/pt)*ceil(H/ph)*ceil(W/pw), and
@@ -242,6 +252,33 @@ veda_status veda_tile_map_workspace(const veda_problem* p, int32_t R, size_t* by
 veda_status veda_tile_map_maxpool(const veda_problem* p, const void* qp, const void* kp,
                                   const int32_t* rows, int32_t R, float scale, float* map,
                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------- training the estimator */
+
+/* Bytes of workspace veda_distill_loss_grad needs. */
+veda_status veda_distill_workspace(const veda_problem* p, int32_t hidden, int32_t e, int32_t R, size_t* bytes);
+
+/* The estimator's distillation objective and its gradients (section 2.1,
+ * "Optimization": a row-wise KL divergence aligns the predicted tile-score
+ * distribution with the full-attention reference; the backbone features fed
+ * to the estimator are stop-gradient).  With the subset rows and tile map of
+ * veda_tile_map_maxpool (map [B, heads, R, NT_max] fp32, rows [B*heads, R]
+ * int32, -1 = unused) and s[i, j] = <phi_q(i), phi_k(j)> / sqrt(e):
+ *   loss = mean over valid subset rows (b, h, r), i = rows[b*heads+h, r], of
+ *          KL(T || P),  T = map[b, h, r, :NT_h] / sum_j map[b, h, r, j],
+ *                       P = softmax_j s[i, j], j < NT_h;
+ *   grad_q / grad_k = d loss / d (W1, b1, W2, b2) of the Q-side and K-side
+ *          estimators; the descriptors get no gradient.
+ * loss: one DEVICE fp32.  When mlp_q and mlp_k are the same weights, their
+ * gradient is grad_q + grad_k.  desc_q, desc_k as for veda_tile_score_topk.
+ * Map rows must have a positive sum.  workspace: >= veda_distill_workspace()
+ * bytes of device scratch, 256-byte aligned.  The forward estimator runs on
+ * the tensor cores as in veda_tile_score_topk; the backward runs in fp32. */
+veda_status veda_distill_loss_grad(const veda_problem* p, const float* desc_q, const float* desc_k,
+                                   const veda_mlp* mlp_q, const veda_mlp* mlp_k, const float* map,
+                                   const int32_t* rows, int32_t R, float* loss, const veda_mlp_grad* grad_q,
+                                   const veda_mlp_grad* grad_k, void* workspace, size_t workspace_bytes,
+                                   void* stream);
 
 /* ---------------------------------------------------------------- status */
 

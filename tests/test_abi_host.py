@@ -123,3 +123,33 @@ def test_attention_config_query(V):
     assert V.veda_attn_config(p64, 2)[:2] == (4, 4)
     with pytest.raises(V.VedaError):
         V.veda_attn_config(p, 0)
+
+
+def test_distill_entry_points_validate_on_the_host(V):
+    B = V.binding
+    p = V.Problem(1, 2, 64, 64, (4, 8, 8), [(1, 8, 8), (4, 4, 4)])
+    nt = p.nt_max
+    # workspace: phi + hidden + dL/ds + row losses + dphi (+ count), each rounded to 256 bytes
+    r256 = lambda x: (x + 255) // 256 * 256
+    bh, hidden, e, R = 2, 128, 32, 3
+    expect = (r256(4 * 2 * bh * nt * e) + r256(4 * 2 * bh * nt * hidden) + r256(4 * bh * R * nt) + r256(4 * bh * R)
+              + r256(4 * 2 * bh * nt * e) + 256)
+    assert V.veda_distill_workspace(p, hidden, e, R) == expect
+    with pytest.raises(V.VedaError):
+        V.veda_distill_workspace(p, hidden, 24, R)     # e not in {16, 32, 64, 128}
+    with pytest.raises(V.VedaError):
+        V.veda_distill_workspace(p, hidden, e, 0)
+    lib = V.LIB
+    m = B.veda_mlp(256, 256, 256, 256, hidden, e)
+    g = B.veda_mlp_grad(256, 256, 256, 256)
+    ok_ws = 4096
+    # NULL tensors, a misaligned workspace and a short workspace are refused before any launch
+    assert lib.veda_distill_loss_grad(p.ref, None, 256, ctypes.byref(m), ctypes.byref(m), 256, 256, R, 256,
+                                      ctypes.byref(g), ctypes.byref(g), ok_ws, 1 << 30, None) == B.VEDA_ERR_INVALID_ARG
+    assert lib.veda_distill_loss_grad(p.ref, 256, 256, ctypes.byref(m), ctypes.byref(m), 256, 256, R, 256,
+                                      ctypes.byref(g), ctypes.byref(g), 4097, 1 << 30, None) == B.VEDA_ERR_INVALID_ARG
+    assert lib.veda_distill_loss_grad(p.ref, 256, 256, ctypes.byref(m), ctypes.byref(m), 256, 256, R, 256,
+                                      ctypes.byref(g), ctypes.byref(g), ok_ws, 16, None) == B.VEDA_ERR_INVALID_ARG
+    bad = B.veda_mlp_grad(256, 0, 256, 256)
+    assert lib.veda_distill_loss_grad(p.ref, 256, 256, ctypes.byref(m), ctypes.byref(m), 256, 256, R, 256,
+                                      ctypes.byref(bad), ctypes.byref(g), ok_ws, 1 << 30, None) == B.VEDA_ERR_INVALID_ARG

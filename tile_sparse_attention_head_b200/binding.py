@@ -48,6 +48,10 @@ class veda_mlp(ctypes.Structure):
                 ("hidden", ctypes.c_int32), ("e", ctypes.c_int32)]
 
 
+class veda_mlp_grad(ctypes.Structure):
+    _fields_ = [("w1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("w2", ctypes.c_void_p), ("b2", ctypes.c_void_p)]
+
+
 _P = ctypes.POINTER(veda_problem)
 _V = ctypes.c_void_p
 _I32P = ctypes.POINTER(ctypes.c_int32)
@@ -69,6 +73,10 @@ _SIG = {
     "veda_attn_config": [_P, ctypes.c_int32, _I32P, _I32P, ctypes.POINTER(ctypes.c_size_t)],
     "veda_tile_map_workspace": [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)],
     "veda_tile_map_maxpool": [_P, _V, _V, _V, ctypes.c_int32, ctypes.c_float, _V, _V, ctypes.c_size_t, _V],
+    "veda_distill_workspace": [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)],
+    "veda_distill_loss_grad": [_P, _V, _V, ctypes.POINTER(veda_mlp), ctypes.POINTER(veda_mlp), _V, _V, ctypes.c_int32,
+                               _V, ctypes.POINTER(veda_mlp_grad), ctypes.POINTER(veda_mlp_grad), _V, ctypes.c_size_t,
+                               _V],
     "veda_sync_status": [_V],
     "veda_set_wait_timeout_ns": [ctypes.c_uint64],
     "veda_selftest_wait_timeout": [ctypes.c_uint64, _V],
@@ -298,6 +306,35 @@ def veda_tile_map_maxpool(p: Problem, qp: torch.Tensor, kp: torch.Tensor, rows: 
         _ptr(out, "map", torch.float32, (p.B, p.heads, R, p.nt_max)), _ptr(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream)), "veda_tile_map_maxpool")
     return out
+
+
+def veda_distill_workspace(p: Problem, hidden: int, e: int, R: int) -> int:
+    n = ctypes.c_size_t()
+    _check(LIB.veda_distill_workspace(p.ref, int(hidden), int(e), int(R), ctypes.byref(n)), "veda_distill_workspace")
+    return int(n.value)
+
+
+def make_mlp_grad(w1: torch.Tensor, b1: torch.Tensor, w2: torch.Tensor, b2: torch.Tensor) -> veda_mlp_grad:
+    """C struct of gradient outputs for one estimator (fp32 device tensors shaped like its weights)."""
+    for t, n in ((w1, "w1"), (b1, "b1"), (w2, "w2"), (b2, "b2")):
+        _ptr(t, n, torch.float32)
+    return veda_mlp_grad(w1.data_ptr(), b1.data_ptr(), w2.data_ptr(), b2.data_ptr())
+
+
+def veda_distill_loss_grad(p: Problem, desc_q: torch.Tensor, desc_k: torch.Tensor, mlp_q: veda_mlp, mlp_k: veda_mlp,
+                           tile_map: torch.Tensor, rows: torch.Tensor, loss: torch.Tensor, grad_q: veda_mlp_grad,
+                           grad_k: veda_mlp_grad, workspace: torch.Tensor, stream=None) -> torch.Tensor:
+    """Row-wise KL distillation loss of the estimator against the tile map, and its gradients."""
+    dshape = (p.B, p.heads, p.nt_max, 3 * p.d)
+    R = int(rows.shape[-1])
+    _check(LIB.veda_distill_loss_grad(
+        p.ref, _ptr(desc_q, "desc_q", torch.float32, dshape), _ptr(desc_k, "desc_k", torch.float32, dshape),
+        ctypes.byref(mlp_q), ctypes.byref(mlp_k),
+        _ptr(tile_map, "map", torch.float32, (p.B, p.heads, R, p.nt_max)),
+        _ptr(rows, "rows", torch.int32, (p.B * p.heads, R)), R, _ptr(loss, "loss", torch.float32, (1,)),
+        ctypes.byref(grad_q), ctypes.byref(grad_k), _ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "veda_distill_loss_grad")
+    return loss
 
 
 def veda_sync_status(stream=None) -> None:

@@ -70,7 +70,7 @@ template <int E>
 __global__ void __launch_bounds__(kEstThreads, 1)
     estimator_kernel(const __grid_constant__ Geometry G, const float* __restrict__ desc_q,
                      const float* __restrict__ desc_k, EstimatorWeights wq, EstimatorWeights wk, int hidden,
-                     float* __restrict__ phi, uint64_t timeout_ns) {
+                     float* __restrict__ phi, float* __restrict__ hid_out, uint64_t timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kEstStage);   // [0,1] stage free, [2] layer done, [3] drain
@@ -182,6 +182,10 @@ __global__ void __launch_bounds__(kEstThreads, 1)
         float v[32];
         tmem_ld32(tmem + kEstAcc1 + ((uint32_t)(warp * 32) << 16) + (uint32_t)(pi * 32), v);
         tmem_ld_wait();
+        // optional copy of the hidden activations [2, B*heads, NT_max, hidden]
+        float* hrow = (hid_out != nullptr && r < nrows)
+                          ? hid_out + (((long long)which * G.B * G.heads + bh) * G.ntmax + j0 + r) * hidden
+                          : nullptr;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           float4 hv;
@@ -191,6 +195,7 @@ __global__ void __launch_bounds__(kEstThreads, 1)
             const int unit = u0 + c * 4 + q;
             hp[q] = (unit < hidden) ? fmaxf(v[c * 4 + q] + __ldg(B1 + unit), 0.f) : 0.f;
           }
+          if (hrow != nullptr && u0 + c * 4 < hidden) *reinterpret_cast<float4*>(hrow + u0 + c * 4) = hv;
           store_split4(ahi, alo, r, c, hv);
         }
       } else {
@@ -266,24 +271,24 @@ __global__ void __launch_bounds__(kEstThreads, 1)
 
 template <int E>
 static cudaError_t launch_est_t(const Geometry& G, const float* dq, const float* dk, const EstimatorWeights& wq,
-                                const EstimatorWeights& wk, int hidden, float* phi, uint64_t timeout_ns,
+                                const EstimatorWeights& wk, int hidden, float* phi, float* hid, uint64_t timeout_ns,
                                 cudaStream_t s) {
   const size_t smem = estimator_smem_bytes(G.d, hidden, E);
   cudaError_t err = cudaFuncSetAttribute(estimator_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid((G.ntmax + kEstRows - 1) / kEstRows, G.B * G.heads, 2);
-  estimator_kernel<E><<<grid, kEstThreads, smem, s>>>(G, dq, dk, wq, wk, hidden, phi, timeout_ns);
+  estimator_kernel<E><<<grid, kEstThreads, smem, s>>>(G, dq, dk, wq, wk, hidden, phi, hid, timeout_ns);
   return cudaGetLastError();
 }
 
 cudaError_t launch_estimator(const Geometry& G, const float* dq, const float* dk, const EstimatorWeights& wq,
-                             const EstimatorWeights& wk, int hidden, int e, float* phi, uint64_t timeout_ns,
-                             cudaStream_t s) {
+                             const EstimatorWeights& wk, int hidden, int e, float* phi, float* hid,
+                             uint64_t timeout_ns, cudaStream_t s) {
   switch (e) {
-    case 16: return launch_est_t<16>(G, dq, dk, wq, wk, hidden, phi, timeout_ns, s);
-    case 32: return launch_est_t<32>(G, dq, dk, wq, wk, hidden, phi, timeout_ns, s);
-    case 64: return launch_est_t<64>(G, dq, dk, wq, wk, hidden, phi, timeout_ns, s);
-    case 128: return launch_est_t<128>(G, dq, dk, wq, wk, hidden, phi, timeout_ns, s);
+    case 16: return launch_est_t<16>(G, dq, dk, wq, wk, hidden, phi, hid, timeout_ns, s);
+    case 32: return launch_est_t<32>(G, dq, dk, wq, wk, hidden, phi, hid, timeout_ns, s);
+    case 64: return launch_est_t<64>(G, dq, dk, wq, wk, hidden, phi, hid, timeout_ns, s);
+    case 128: return launch_est_t<128>(G, dq, dk, wq, wk, hidden, phi, hid, timeout_ns, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -65,8 +65,8 @@ cudaError_t launch_tripool(const Geometry& G, const void* xp, float* desc, cudaS
 
 size_t estimator_smem_bytes(int d, int hidden, int e);
 cudaError_t launch_estimator(const Geometry& G, const float* dq, const float* dk, const EstimatorWeights& wq,
-                             const EstimatorWeights& wk, int hidden, int e, float* phi, uint64_t timeout_ns,
-                             cudaStream_t s);
+                             const EstimatorWeights& wk, int hidden, int e, float* phi, float* hid,
+                             uint64_t timeout_ns, cudaStream_t s);
 void score_topk_config(int ntmax, int e, int* qb, int* ntpad, size_t* smem);
 cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const float* desc_k,
                               const EstimatorWeights& wq, const EstimatorWeights& wk, int hidden,
@@ -85,6 +85,12 @@ cudaError_t launch_tripool_grid(const Geometry& G, const void* x, float* desc, c
 
 cudaError_t launch_tile_map(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,
                             const MapArgs& a, cudaStream_t s);
+
+size_t distill_ws_bytes(const Geometry& G, int hidden, int e, int R);
+cudaError_t launch_distill(const Geometry& G, const float* desc_q, const float* desc_k, const EstimatorWeights& wq,
+                           const EstimatorWeights& wk, int hidden, int e, const float* map, const int32_t* rows,
+                           int R, float* loss, const EstimatorWeights& gq, const EstimatorWeights& gk, void* ws,
+                           uint64_t timeout_ns, cudaStream_t s);
 
 cudaError_t launch_timeout_selftest(uint64_t timeout_ns, cudaStream_t s);
 

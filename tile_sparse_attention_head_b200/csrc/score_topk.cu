@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kScoreThreads)
 cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const float* desc_k,
                               const EstimatorWeights& wq, const EstimatorWeights& wk, int hidden,
                               int e, float* phi, const TopkArgs& args, cudaStream_t s) {
-  cudaError_t err = launch_estimator(G, desc_q, desc_k, wq, wk, hidden, e, phi, args.timeout_ns, s);
+  cudaError_t err = launch_estimator(G, desc_q, desc_k, wq, wk, hidden, e, phi, nullptr, args.timeout_ns, s);
   if (err != cudaSuccess) return err;
 
   int qb, ntpad;

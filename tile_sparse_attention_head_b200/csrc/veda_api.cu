@@ -19,6 +19,7 @@
 #include "score_topk.cu"
 #include "sparse_attn.cu"
 #include "tile_map.cu"
+#include "distill.cu"
 
 namespace veda {
 namespace {
@@ -568,6 +569,56 @@ veda_status veda_tile_map_maxpool(const veda_problem* p, const void* qp, const v
   a.timeout_ns = g_timeout_ns;
   cudaError_t e = launch_tile_map(G, tq, tk, a, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "veda_tile_map_maxpool");
+  return ok();
+}
+
+veda_status veda_distill_workspace(const veda_problem* p, int32_t hidden, int32_t e, int32_t R, size_t* bytes) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (hidden < 4 || hidden > 512 || hidden % 4) return fail(VEDA_ERR_INVALID_ARG, "hidden must be a multiple of 4 in [4, 512]");
+  if (e != 16 && e != 32 && e != 64 && e != 128) return fail(VEDA_ERR_INVALID_ARG, "e must be 16, 32, 64 or 128 (got %d)", e);
+  if (R < 1) return fail(VEDA_ERR_INVALID_ARG, "R must be >= 1 (got %d)", R);
+  if (!bytes) return fail(VEDA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = distill_ws_bytes(G, hidden, e, R);
+  return ok();
+}
+
+veda_status veda_distill_loss_grad(const veda_problem* p, const float* desc_q, const float* desc_k,
+                                   const veda_mlp* mlp_q, const veda_mlp* mlp_k, const float* map,
+                                   const int32_t* rows, int32_t R, float* loss, const veda_mlp_grad* grad_q,
+                                   const veda_mlp_grad* grad_k, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if ((s = check_mlp(mlp_q, "q")) != VEDA_OK || (s = check_mlp(mlp_k, "k")) != VEDA_OK) return s;
+  if (mlp_q->hidden != mlp_k->hidden || mlp_q->e != mlp_k->e)
+    return fail(VEDA_ERR_INVALID_ARG, "q and k estimators must have the same hidden and e");
+  if (R < 1) return fail(VEDA_ERR_INVALID_ARG, "R must be >= 1 (got %d)", R);
+  if (!desc_q || !desc_k || !map || !rows || !loss || !grad_q || !grad_k || !workspace)
+    return fail(VEDA_ERR_INVALID_ARG, "NULL argument");
+  const veda_mlp_grad* gs[2] = {grad_q, grad_k};
+  for (const veda_mlp_grad* g : gs) {
+    if (!g->w1 || !g->b1 || !g->w2 || !g->b2) return fail(VEDA_ERR_INVALID_ARG, "NULL gradient pointer");
+    if (!aligned16(g->w1) || !aligned16(g->b1) || !aligned16(g->w2) || !aligned16(g->b2))
+      return fail(VEDA_ERR_INVALID_ARG, "gradient pointers must be 16-byte aligned");
+  }
+  if (!aligned16(desc_q) || !aligned16(desc_k) || !aligned16(map) || !aligned16(rows) || !aligned16(loss))
+    return fail(VEDA_ERR_INVALID_ARG, "tensor arguments must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(VEDA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const int e = mlp_q->e, hidden = mlp_q->hidden;
+  if (workspace_bytes < distill_ws_bytes(G, hidden, e, R))
+    return fail(VEDA_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu required", workspace_bytes,
+                distill_ws_bytes(G, hidden, e, R));
+  EstimatorWeights wq{mlp_q->w1, mlp_q->b1, mlp_q->w2, mlp_q->b2};
+  EstimatorWeights wk{mlp_k->w1, mlp_k->b1, mlp_k->w2, mlp_k->b2};
+  EstimatorWeights gq{grad_q->w1, grad_q->b1, grad_q->w2, grad_q->b2};
+  EstimatorWeights gk{grad_k->w1, grad_k->b1, grad_k->w2, grad_k->b2};
+  cudaError_t ce = launch_distill(G, desc_q, desc_k, wq, wk, hidden, e, map, rows, R, loss, gq, gk, workspace,
+                                  g_timeout_ns, (cudaStream_t)stream);
+  if (ce != cudaSuccess) return cuda_fail(ce, "veda_distill_loss_grad");
   return ok();
 }
 
