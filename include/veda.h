@@ -280,6 +280,18 @@ veda_status veda_distill_loss_grad(const veda_problem* p, const float* desc_q, c
                                    const veda_mlp_grad* grad_k, void* workspace, size_t workspace_bytes,
                                    void* stream);
 
+/* ---------------------------------------------------------------- offline tiling search */
+
+/* Per-head error between two grid-order outputs, for the offline choice of
+ * each head's tiling (section 2.2: the tiling is selected on a calibration
+ * set by minimising the error between full- and sparse-attention outputs).
+ * o, o_ref [B, heads, N, d] bf16 (read).  err[h] = sum over b, n, channels
+ * of (o - o_ref)^2 and ref_sq[h] = sum of o_ref^2; both DEVICE fp32 [heads],
+ * written in full, summed in a fixed order.  workspace: >= 512 * heads bytes
+ * of device scratch, 16-byte aligned. */
+veda_status veda_head_error(const veda_problem* p, const void* o, const void* o_ref, float* err, float* ref_sq,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------------------- status */
 
 /* Synchronises `stream`, then reads and clears the library's device error

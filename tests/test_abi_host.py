@@ -153,3 +153,12 @@ def test_distill_entry_points_validate_on_the_host(V):
     bad = B.veda_mlp_grad(256, 0, 256, 256)
     assert lib.veda_distill_loss_grad(p.ref, 256, 256, ctypes.byref(m), ctypes.byref(m), 256, 256, R, 256,
                                       ctypes.byref(bad), ctypes.byref(g), ok_ws, 1 << 30, None) == B.VEDA_ERR_INVALID_ARG
+
+
+def test_head_error_validates_on_the_host(V):
+    B = V.binding
+    p = V.Problem(1, 2, 64, 64, (4, 8, 8), [(1, 8, 8), (4, 4, 4)])
+    lib = V.LIB
+    assert lib.veda_head_error(p.ref, None, 256, 256, 256, 256, 4096, None) == B.VEDA_ERR_INVALID_ARG
+    assert lib.veda_head_error(p.ref, 8, 256, 256, 256, 256, 4096, None) == B.VEDA_ERR_INVALID_ARG
+    assert lib.veda_head_error(p.ref, 256, 256, 256, 256, 256, 16, None) == B.VEDA_ERR_INVALID_ARG   # short workspace

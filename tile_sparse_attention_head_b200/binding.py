@@ -77,6 +77,7 @@ _SIG = {
     "veda_distill_loss_grad": [_P, _V, _V, ctypes.POINTER(veda_mlp), ctypes.POINTER(veda_mlp), _V, _V, ctypes.c_int32,
                                _V, ctypes.POINTER(veda_mlp_grad), ctypes.POINTER(veda_mlp_grad), _V, ctypes.c_size_t,
                                _V],
+    "veda_head_error": [_P, _V, _V, _V, _V, _V, ctypes.c_size_t, _V],
     "veda_sync_status": [_V],
     "veda_set_wait_timeout_ns": [ctypes.c_uint64],
     "veda_selftest_wait_timeout": [ctypes.c_uint64, _V],
@@ -335,6 +336,17 @@ def veda_distill_loss_grad(p: Problem, desc_q: torch.Tensor, desc_k: torch.Tenso
         ctypes.byref(grad_q), ctypes.byref(grad_k), _ptr(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream)), "veda_distill_loss_grad")
     return loss
+
+
+def veda_head_error(p: Problem, o: torch.Tensor, o_ref: torch.Tensor, err: torch.Tensor, ref_sq: torch.Tensor,
+                    workspace: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-head sums of (o - o_ref)^2 and o_ref^2 over grid-order bf16 outputs."""
+    gs = p.grid_shape()
+    _check(LIB.veda_head_error(p.ref, _ptr(o, "o", torch.bfloat16, gs), _ptr(o_ref, "o_ref", torch.bfloat16, gs),
+                               _ptr(err, "err", torch.float32, (p.heads,)),
+                               _ptr(ref_sq, "ref_sq", torch.float32, (p.heads,)), _ptr(workspace, "workspace"),
+                               workspace.numel() * workspace.element_size(), _stream(stream)), "veda_head_error")
+    return err, ref_sq
 
 
 def veda_sync_status(stream=None) -> None:

@@ -303,6 +303,64 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Per-head output error for the offline tiling search (section 2.2: a head's
+// tiling is chosen to minimise the error between full and sparse attention
+// outputs): err[h] = sum_{b, n, c} (o - o_ref)^2 and ref[h] = sum o_ref^2 over
+// grid-order bf16 tensors [B, heads, N, d].  grid (blocks_per_head, heads);
+// each CTA writes one partial pair, summed in a fixed order by
+// head_error_finish_kernel.
+__global__ void __launch_bounds__(256) head_error_kernel(const __grid_constant__ Geometry G,
+                                                         const uint4* __restrict__ o, const uint4* __restrict__ o_ref,
+                                                         float* __restrict__ part) {
+  __shared__ float red[32];
+  const int h = blockIdx.y;
+  const long long per_bh = (long long)G.N * G.d / 8;   // 16-byte chunks per (b, h)
+  float se = 0.f, sr = 0.f;
+  for (int b = 0; b < G.B; ++b) {
+    const uint4* x = o + ((long long)b * G.heads + h) * per_bh;
+    const uint4* y = o_ref + ((long long)b * G.heads + h) * per_bh;
+    for (long long c = blockIdx.x * 256LL + threadIdx.x; c < per_bh; c += (long long)gridDim.x * 256) {
+      const uint4 u = __ldg(x + c), v = __ldg(y + c);
+      const __nv_bfloat162* pu = reinterpret_cast<const __nv_bfloat162*>(&u);
+      const __nv_bfloat162* pv = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 a = __bfloat1622float2(pu[k]), r = __bfloat1622float2(pv[k]);
+        se = fmaf(a.x - r.x, a.x - r.x, fmaf(a.y - r.y, a.y - r.y, se));
+        sr = fmaf(r.x, r.x, fmaf(r.y, r.y, sr));
+      }
+    }
+  }
+  se = block_reduce_sum(se, red);
+  sr = block_reduce_sum(sr, red);
+  if (threadIdx.x == 0) {
+    part[((long long)h * gridDim.x + blockIdx.x) * 2 + 0] = se;
+    part[((long long)h * gridDim.x + blockIdx.x) * 2 + 1] = sr;
+  }
+}
+
+__global__ void head_error_finish_kernel(const float* __restrict__ part, int nblk, int heads, float* __restrict__ err,
+                                         float* __restrict__ ref) {
+  for (int h = threadIdx.x; h < heads; h += blockDim.x) {
+    float se = 0.f, sr = 0.f;
+    for (int k = 0; k < nblk; ++k) {
+      se += part[((long long)h * nblk + k) * 2 + 0];
+      sr += part[((long long)h * nblk + k) * 2 + 1];
+    }
+    err[h] = se;
+    ref[h] = sr;
+  }
+}
+
+constexpr int kHeadErrBlocks = 64;   // partial sums per head
+
+cudaError_t launch_head_error(const Geometry& G, const void* o, const void* o_ref, float* err, float* ref,
+                              float* part, cudaStream_t s) {
+  head_error_kernel<<<dim3(kHeadErrBlocks, G.heads), 256, 0, s>>>(G, (const uint4*)o, (const uint4*)o_ref, part);
+  head_error_finish_kernel<<<1, 128, 0, s>>>(part, kHeadErrBlocks, G.heads, err, ref);
+  return cudaGetLastError();
+}
+
 size_t distill_ws_bytes(const Geometry& G, int hidden, int e, int R) {
   const size_t BH = (size_t)G.B * G.heads, nt = (size_t)G.ntmax;
   auto r256 = [](size_t x) { return (x + 255) & ~size_t(255); };

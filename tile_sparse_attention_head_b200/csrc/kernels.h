@@ -87,6 +87,8 @@ cudaError_t launch_tile_map(const Geometry& G, const CUtensorMap& tq, const CUte
                             const MapArgs& a, cudaStream_t s);
 
 size_t distill_ws_bytes(const Geometry& G, int hidden, int e, int R);
+cudaError_t launch_head_error(const Geometry& G, const void* o, const void* o_ref, float* err, float* ref,
+                              float* part, cudaStream_t s);
 cudaError_t launch_distill(const Geometry& G, const float* desc_q, const float* desc_k, const EstimatorWeights& wq,
                            const EstimatorWeights& wk, int hidden, int e, const float* map, const int32_t* rows,
                            int R, float* loss, const EstimatorWeights& gq, const EstimatorWeights& gk, void* ws,

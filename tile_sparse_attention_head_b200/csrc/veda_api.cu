@@ -622,6 +622,21 @@ veda_status veda_distill_loss_grad(const veda_problem* p, const float* desc_q, c
   return ok();
 }
 
+veda_status veda_head_error(const veda_problem* p, const void* o, const void* o_ref, float* err, float* ref_sq,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (!o || !o_ref || !err || !ref_sq || !workspace) return fail(VEDA_ERR_INVALID_ARG, "NULL argument");
+  if (!aligned16(o) || !aligned16(o_ref) || !aligned16(workspace))
+    return fail(VEDA_ERR_INVALID_ARG, "tensor arguments must be 16-byte aligned");
+  const size_t need = sizeof(float) * 2 * (size_t)kHeadErrBlocks * G.heads;
+  if (workspace_bytes < need) return fail(VEDA_ERR_INVALID_ARG, "workspace needs %zu bytes", need);
+  cudaError_t ce = launch_head_error(G, o, o_ref, err, ref_sq, static_cast<float*>(workspace), (cudaStream_t)stream);
+  if (ce != cudaSuccess) return cuda_fail(ce, "veda_head_error");
+  return ok();
+}
+
 veda_status veda_sync_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "veda_sync_status: stream synchronize");
