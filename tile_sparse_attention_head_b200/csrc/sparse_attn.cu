@@ -24,8 +24,8 @@
 //                row sum) and its own O accumulator, so the two warps that
 //                share a scheduler work on different tiles and never wait for
 //                each other; a thread owns one query row (its TMEM lane) and
-//                all BN columns of it.  Exponentials run in the log2 domain,
-//                a share of them on the FMA pipe; O is rescaled in TMEM only
+//                all BN columns of it.  Exponentials run in the log2 domain on
+//                the special-function unit; O is rescaled in TMEM only
 //                when the stream's maximum grows by more than 2^8; P is
 //                written as packed bf16 to the stream's own P buffer.
 //                At the end the two partial results are merged exactly:
@@ -40,10 +40,11 @@
 
 namespace veda {
 
-// Three pairs of exponentials in eight are evaluated with exp2_fma_x2 (FMA
-// pipe), the others with ex2.approx (special-function unit, a quarter of the
-// FMA rate): this balances the two pipes of a row of 128 scores.
-__host__ __device__ constexpr bool poly_pair(int pair) { return (pair * 3) % 8 < 3; }
+// Every exponential runs on the special-function unit (ex2.approx).  The
+// kernel runs at the board's power cap, where throughput follows energy per
+// tile: moving a share of the exponentials to an FMA-pipe polynomial
+// balances the pipes but costs more instructions, and measured at sustained
+// load it is slower (1/8 of them: -3%, 3/8: -9%).
 constexpr int kSmemLimit = 232448;   // dynamic shared memory per CTA on sm_100
 
 // Shared memory: the bookkeeping (barriers, the final (m, l) exchange, flags,
@@ -442,8 +443,8 @@ __global__ void __launch_bounds__(384, 1)
         m_use = m_run;
       }
       const float m_ref = (m_use == -INFINITY) ? 0.f : m_use;
-      // x = s*scale*log2(e) - m_ref as packed pairs; every kPolyEvery-th pair
-      // of exponentials on the FMA pipe; row sum over 4 packed chains.
+      // x = s*scale*log2(e) - m_ref as packed pairs; row sum over 4 packed
+      // chains.
       const uint64_t scl2 = f2(sl2, sl2), nref2 = f2(-m_ref, -m_ref);
       uint64_t r4[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[BN / 2];
@@ -451,12 +452,8 @@ __global__ void __launch_bounds__(384, 1)
       for (int c = 0; c < BN; c += 2) {
         float x0, x1, p0, p1;
         f2_split(f2_fma(f2(sc[c], sc[c + 1]), scl2, nref2), x0, x1);
-        if (poly_pair(c >> 1)) {
-          exp2_fma_x2(x0, x1, p0, p1);
-        } else {
-          p0 = fast_exp2(x0);
-          p1 = fast_exp2(x1);
-        }
+        p0 = fast_exp2(x0);
+        p1 = fast_exp2(x1);
         r4[(c >> 1) & 3] = f2_add(r4[(c >> 1) & 3], f2(p0, p1));
         pk[c >> 1] = pack_bf16x2(p0, p1);
       }

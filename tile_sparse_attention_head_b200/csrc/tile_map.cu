@@ -27,10 +27,11 @@
 
 namespace veda {
 
-// Pass 1 is exponential-bound (Q K^T only): three pairs of exponentials in
-// eight run on the FMA pipe (exp2_fma_x2), the rest on the special-function
-// unit.
-__host__ __device__ constexpr bool map_poly_pair(int pair) { return (pair * 3) % 8 < 3; }
+// Pass 1 is exponential-bound (Q K^T only): one pair of exponentials in
+// eight runs on the FMA pipe (exp2_fma_x2), the rest on the special-function
+// unit.  At the board's power cap this split measured fastest (10.1 ms at
+// the 14B shape against 10.4 with none and 10.9 with 3/8 on the FMA pipe).
+__host__ __device__ constexpr bool map_poly_pair(int pair) { return pair % 8 == 7; }
 
 template <int D, int BN>
 struct MapCfg {
