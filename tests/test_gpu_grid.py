@@ -188,3 +188,21 @@ def test_extreme_score_in_the_last_key_slot(V):
     assert ref_l[0, 0, 0] > 150.0                               # the extreme row really is extreme
     check_attn_rows(g[0, 0], ref_o[0, 0])
     assert np.abs(gl[0, 0] - ref_l[0, 0]).max() <= LSE_ABS
+
+
+def test_host_buffer_pipeline_equals_the_device_path(V):
+    """VedaAttentionHost (head chunks pipelined over three streams, pinned host
+    buffers) gives exactly the device-resident layer's output, B = 2 included."""
+    w = SMALL[2]                                      # odd128: B = 2, 4 heads
+    p = _problem(V, w)
+    q, k, v = make_qkv(w, seed=3)
+    md = mlp_device(make_mlp(w, seed=1))
+    ref = V.VedaAttention(p, md, md, w.keep, layout="grid")(q.cuda(), k.cuda(), v.cuda())
+    host = V.VedaAttentionHost(p, md, md, w.keep, chunk_heads=3, slots=2)
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.full(p.grid_shape(), float("nan"), dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):                                # slot reuse across calls
+        host(qh, kh, vh, oh)
+        torch.cuda.synchronize()
+        V.veda_sync_status()
+        assert torch.equal(oh, ref.cpu())

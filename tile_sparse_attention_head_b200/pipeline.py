@@ -90,3 +90,80 @@ class VedaAttention:
         else:
             B.veda_tile_sparse_attn_grid(p, q, k, v, self.idx, out, self.lse, 0.0, stream)
         return out
+
+
+class VedaAttentionHost:
+    """The layer on HOST buffers: pinned grid-order bf16 Q, K, V in, O out.
+
+    Every (b, head) is independent through all steps, so the heads are cut
+    into chunks and the chunks are pipelined over three CUDA streams: while
+    chunk c is attended, chunk c+1's Q/K/V are copied in and chunk c-1's
+    output is copied out (PCIe is full duplex, so both directions run at
+    once).  ``slots`` device buffer sets rotate between the chunks.  Every
+    compute step is the library's (one VedaAttention per chunk, grid-order
+    layout); the copies are cudaMemcpyAsync from pinned memory.
+    """
+
+    def __init__(self, problem: B.Problem, mlp_q, mlp_k, keep_ratio: float, device="cuda", chunk_heads: int = 5,
+                 slots: int = 3):
+        p = problem
+        self.p = p
+        self.dev = torch.device(device)
+        self.chunks = []                       # (b, h0, h1, slot index, VedaAttention)
+        ch = max(1, int(chunk_heads))
+        n = 0
+        for b in range(p.B):
+            for h0 in range(0, p.heads, ch):
+                h1 = min(p.heads, h0 + ch)
+                sub = B.Problem(1, h1 - h0, p.d, p.S, p.grid, p.tilings[h0:h1])
+                mq = tuple(t[h0:h1] for t in mlp_q)
+                mk = tuple(t[h0:h1] for t in mlp_k)
+                self.chunks.append((b, h0, h1, n % slots, VedaAttention(sub, mq, mk, keep_ratio, device=self.dev)))
+                n += 1
+        self.slots = min(slots, n)
+        rows = min(ch, p.heads) * p.N * p.d
+        self.buf = [[torch.empty(rows, dtype=torch.bfloat16, device=self.dev) for _ in range(4)]
+                    for _ in range(self.slots)]
+        self.s_in, self.s_run, self.s_out = (torch.cuda.Stream(device=self.dev) for _ in range(3))
+
+    def __call__(self, q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor, out_host: torch.Tensor,
+                 stream=None) -> torch.Tensor:
+        """Enqueues the layer after the work already on ``stream`` (default: the
+        current stream) and makes ``stream`` wait for its end; out_host is
+        complete once ``stream`` reaches that point."""
+        p = self.p
+        shape = p.grid_shape()
+        for t, n in ((q_host, "q"), (k_host, "k"), (v_host, "v"), (out_host, "out")):
+            if tuple(t.shape) != shape or t.dtype != torch.bfloat16 or t.is_cuda or not t.is_pinned():
+                raise ValueError(f"{n} must be a pinned host bf16 tensor of shape {shape}")
+        base = stream if stream is not None else torch.cuda.current_stream(self.dev)
+        start = torch.cuda.Event()
+        start.record(base)
+        for s in (self.s_in, self.s_run, self.s_out):
+            s.wait_event(start)
+        free = [None] * self.slots             # slot reusable once its output is copied out
+        last = None
+        for b, h0, h1, slot, att in self.chunks:
+            qb, kb, vb, ob = self.buf[slot]
+            n = (h1 - h0) * p.N * p.d
+            gshape = (1, h1 - h0, p.N, p.d)
+            with torch.cuda.stream(self.s_in):
+                if free[slot] is not None:
+                    self.s_in.wait_event(free[slot])
+                for dst, src in ((qb, q_host), (kb, k_host), (vb, v_host)):
+                    dst[:n].view(gshape).copy_(src[b:b + 1, h0:h1], non_blocking=True)
+                loaded = torch.cuda.Event()
+                loaded.record(self.s_in)
+            self.s_run.wait_event(loaded)
+            att(qb[:n].view(gshape), kb[:n].view(gshape), vb[:n].view(gshape), ob[:n].view(gshape),
+                stream=self.s_run)
+            done = torch.cuda.Event()
+            done.record(self.s_run)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(done)
+                out_host[b:b + 1, h0:h1].copy_(ob[:n].view(gshape), non_blocking=True)
+                last = torch.cuda.Event()
+                last.record(self.s_out)
+            free[slot] = last
+        base.wait_event(last)
+        return out_host
