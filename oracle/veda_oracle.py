@@ -269,6 +269,69 @@ def sparse_attention(qp, kp, vp, idx, grid, tilings, S, scale=None):
 
 
 # --------------------------------------------------------------------------
+# Backward of step 5 -- gradients of the tile-skipping attention with respect
+# to Q, K and V, over the selected tiles only.  The pages train only the
+# estimator (section 2.1, "Optimization"); this is the chain rule through the
+# forward defined above, for callers that fine-tune the backbone with the
+# sparse pattern fixed.
+# --------------------------------------------------------------------------
+def attention_tile_backward(qp_h, kp_h, vp_h, dop_h, table, i, sel, S, scale):
+    """Gradient contributions of Q tile i of one head.
+
+    With X = scale * Q K^T over every valid key slot of the selected tiles
+    (the rows of attention_tile), P = softmax over each row of X and O = P V,
+    an upstream gradient dO gives
+        dV = P^T dO,   dP = dO V^T,   dX = P * (dP - rowsum(P * dP)),
+        dQ = scale * dX K,   dK = scale * dX^T Q.
+    Returns (dq [S, d] with pad query slots zero, key_rows, dk, dv), where
+    key_rows are the permuted rows of the keys used and dk, dv the
+    contributions to those rows.
+    """
+    sel = [int(j) for j in sel if j >= 0]
+    key_rows = np.concatenate([j * S + np.nonzero(table[j * S:(j + 1) * S] >= 0)[0] for j in sel])
+    K = kp_h[key_rows]
+    V = vp_h[key_rows]
+    d = qp_h.shape[1]
+    qslots = np.nonzero(table[i * S:(i + 1) * S] >= 0)[0]
+    Q = qp_h[i * S + qslots]
+    dO = dop_h[i * S + qslots]
+    x = scale * (Q @ K.T)
+    p = np.exp(x - x.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    dv = p.T @ dO
+    dp = dO @ V.T
+    dx = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+    dq = np.zeros((S, d), dtype=np.float64)
+    dq[qslots] = scale * (dx @ K)
+    dk = scale * (dx.T @ Q)
+    return dq, key_rows, dk, dv
+
+
+def sparse_attention_backward(qp, kp, vp, dop, idx, grid, tilings, S, scale=None):
+    """dQp, dKp, dVp [B, heads, NT_max*S, d] (tile-major, pad rows zero) of the
+    tile-skipping attention for the upstream gradient dOp (same layout).
+    A key row's dK and dV sum the contributions of every Q tile that
+    selected its tile."""
+    B, heads, rows, d = qp.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dqp = np.zeros((B, heads, rows, d), dtype=np.float64)
+    dkp = np.zeros_like(dqp)
+    dvp = np.zeros_like(dqp)
+    for h in range(heads):
+        tab = slot_table(grid, tilings[h])
+        nt = tab.size // S
+        for b in range(B):
+            for i in range(nt):
+                dq, kr, dk, dv = attention_tile_backward(qp[b, h], kp[b, h], vp[b, h], dop[b, h], tab, i,
+                                                         idx[b, h, i], S, scale)
+                dqp[b, h, i * S:(i + 1) * S] = dq
+                dkp[b, h, kr] += dk
+                dvp[b, h, kr] += dv
+    return dqp, dkp, dvp
+
+
+# --------------------------------------------------------------------------
 # Secondary path -- max-pooled full-attention tile map (sections 2.1, 2.3).
 # --------------------------------------------------------------------------
 def tile_map_row(qp_h, kp_h, table, i, S, scale):

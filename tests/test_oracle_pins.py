@@ -444,3 +444,113 @@ def test_distill_loss_and_gradients_vanish_when_the_target_is_the_prediction():
     assert abs(loss) < 1e-13
     for g in gq + gk:
         assert np.abs(g).max() < 1e-12
+
+
+# ---------------------------------------------------------------- backward of step 5
+def _bwd_case(grid=(3, 5, 7), tilings=((1, 2, 4), (2, 2, 2)), S=8, d=8, kept=3, seed=11):
+    rng = np.random.default_rng(seed)
+    N = grid[0] * grid[1] * grid[2]
+    q, k, v, do = (rng.standard_normal((1, 2, N, d)) for _ in range(4))
+    nts, ntmax = O.tile_layout(grid, tilings)
+    idx = np.full((1, 2, ntmax, kept + 1), -1, dtype=np.int32)
+    for h, nt in enumerate(nts):
+        for i in range(nt):
+            idx[0, h, i, :kept] = np.sort(rng.choice(nt, kept, replace=False))
+    return grid, list(tilings), S, q, k, v, do, idx
+
+
+def _bwd_grid(grid, tilings, S, q, k, v, do, idx, scale=None):
+    qp, kp, vp, dop = (O.tile_permute(a, grid, tilings, S) for a in (q, k, v, do))
+    return [O.tile_unpermute(g, grid, tilings, S)
+            for g in O.sparse_attention_backward(qp, kp, vp, dop, idx, grid, tilings, S, scale)]
+
+
+def test_attention_backward_matches_central_differences_of_the_forward():
+    """dQ, dK, dV against central differences of L = <O, dO> through the
+    (separately pinned) oracle forward, on every input entry."""
+    grid, tilings, S, q, k, v, do, idx = _bwd_case(grid=(2, 3, 4), tilings=((1, 2, 2), (2, 1, 2)), S=4, d=3,
+                                                   kept=2)
+    dq, dk, dv = _bwd_grid(grid, tilings, S, q, k, v, do, idx)
+
+    def loss(qq, kk, vv):
+        qp, kp, vp = (O.tile_permute(a, grid, tilings, S) for a in (qq, kk, vv))
+        op, _ = O.sparse_attention(qp, kp, vp, idx, grid, tilings, S)
+        return float((O.tile_unpermute(op, grid, tilings, S) * do).sum())
+
+    eps = 1e-6
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        num = np.zeros_like(grad)
+        for pos in np.ndindex(grad.shape):
+            args = [q.copy(), k.copy(), v.copy()]
+            args[which][pos] += eps
+            up = loss(*args)
+            args[which][pos] -= 2 * eps
+            num[pos] = (up - loss(*args)) / (2 * eps)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8)
+
+
+def test_attention_backward_equals_torch_autograd_of_masked_attention():
+    """The same gradients from torch's fp64 autograd through a dense masked
+    softmax attention (query n may see key m iff m's tile is selected by n's
+    tile), built in grid coordinates without the permutation."""
+    grid, tilings, S, q, k, v, do, idx = _bwd_case()
+    dq, dk, dv = _bwd_grid(grid, tilings, S, q, k, v, do, idx)
+    N = grid[0] * grid[1] * grid[2]
+    d = q.shape[-1]
+    for h in range(2):
+        members = box_members(grid, tilings[h])
+        tile_of = np.empty(N, dtype=np.int64)
+        for j, m in enumerate(members):
+            tile_of[m] = j
+        allowed = np.zeros((N, N), dtype=bool)
+        for n in range(N):
+            sel = set(int(j) for j in idx[0, h, tile_of[n]] if j >= 0)
+            allowed[n] = [tile_of[m] in sel for m in range(N)]
+        tq, tk, tv = (torch.tensor(a[0, h], requires_grad=True) for a in (q, k, v))
+        x = (tq @ tk.T) / math.sqrt(d)
+        x = x.masked_fill(~torch.tensor(allowed), float("-inf"))
+        o = torch.softmax(x, dim=-1) @ tv
+        o.backward(torch.tensor(do[0, h]))
+        np.testing.assert_allclose(dq[0, h], tq.grad.numpy(), rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(dk[0, h], tk.grad.numpy(), rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(dv[0, h], tv.grad.numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_attention_backward_at_full_keep_equals_dense_sdpa_autograd():
+    grid, tilings, S = (4, 8, 8), [(1, 8, 8), (4, 4, 4)], 64
+    rng = np.random.default_rng(12)
+    N = 256
+    q, k, v, do = (rng.standard_normal((1, 2, N, 16)) for _ in range(4))
+    nts, ntmax = O.tile_layout(grid, tilings)
+    idx = np.full((1, 2, ntmax, ntmax), -1, dtype=np.int32)
+    for h, nt in enumerate(nts):
+        idx[0, h, :nt, :nt] = np.arange(nt)
+    dq, dk, dv = _bwd_grid(grid, tilings, S, q, k, v, do, idx)
+    tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+    torch.nn.functional.scaled_dot_product_attention(tq, tk, tv).backward(torch.tensor(do))
+    for g, t in ((dq, tq), (dk, tk), (dv, tv)):
+        np.testing.assert_allclose(g, t.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_attention_backward_sum_invariants():
+    """Softmax rows sum to 1 and its gradient rows to 0: summed over all keys,
+    dV equals the sum of dO over the query rows that see at least one key, and
+    dK sums to zero."""
+    grid, tilings, S, q, k, v, do, idx = _bwd_case(seed=13)
+    dq, dk, dv = _bwd_grid(grid, tilings, S, q, k, v, do, idx)
+    for h in range(2):
+        np.testing.assert_allclose(dv[0, h].sum(axis=0), do[0, h].sum(axis=0), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(dk[0, h].sum(axis=0), 0.0, atol=1e-12)
+    assert np.abs(dq).max() > 1e-3 and np.abs(dk).max() > 1e-3
+
+
+def test_attention_backward_scale_enters_dq_and_dk_only_through_the_logits():
+    """With a custom scale c, dQ and dK carry one factor c beyond the logits:
+    scaling Q by c at scale 1 must give dQ_c = c * dQ_1(cQ) and dK_c = dK_1(cQ)."""
+    grid, tilings, S, q, k, v, do, idx = _bwd_case(seed=14)
+    c = 0.37
+    dq_c, dk_c, dv_c = _bwd_grid(grid, tilings, S, q, k, v, do, idx, scale=c)
+    dq_1, dk_1, dv_1 = _bwd_grid(grid, tilings, S, c * q, k, v, do, idx, scale=1.0)
+    np.testing.assert_allclose(dq_c, c * dq_1, rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(dk_c, dk_1, rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(dv_c, dv_1, rtol=1e-11, atol=1e-13)
