@@ -292,6 +292,37 @@ veda_status veda_distill_loss_grad(const veda_problem* p, const float* desc_q, c
 veda_status veda_head_error(const veda_problem* p, const void* o, const void* o_ref, float* err, float* ref_sq,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------- backward of step 5 */
+
+/* Workspace bytes veda_tile_sparse_attn_backward_grid needs for a problem and
+ * k_max: the row sums D, the inverse selection lists and their offsets. */
+veda_status veda_attn_backward_workspace(const veda_problem* p, int32_t k_max, size_t* bytes);
+
+/* Gradients of veda_tile_sparse_attn_grid with respect to q, k and v over
+ * the same selected tiles (section 2.3 defines the forward; this is its chain
+ * rule, for fine-tuning the backbone with the sparse pattern fixed).  With
+ * P = softmax(scale Q K^T) over the selected tiles' token slots:
+ *   dV = P^T dO,  dP = dO V^T,  dX = P (dP - rowsum(dO * O)),
+ *   dQ = scale dX K,  dK = scale dX^T Q,
+ * where a key row's dK and dV sum over every Q tile that selected its tile.
+ * q, k, v, o, d_o [B, heads, N, d] bf16 grid order (read): the forward's
+ * inputs, its output o and the upstream gradient.  lse [B, heads, N] fp32
+ * (read): the forward's LSE (required).  idx, k_max and scale as given to the
+ * forward (rows read up to their first entry outside [0, NT_h); entries
+ * distinct).  dq, dk, dv [B, heads, N, d] bf16 (written, every row; rows of
+ * keys that no Q tile selected get zero).  They must not overlap the inputs.
+ * workspace: device memory of veda_attn_backward_workspace bytes, 256-byte
+ * aligned, owned by the caller; its contents need no initialisation.  Runs on
+ * the tcgen05 tensor cores with fp32 accumulation; P and dS are rounded to
+ * bf16 as product operands, as in the forward.  Deterministic: no atomics on
+ * the gradients.  Errors: VEDA_ERR_INVALID_ARG for NULL or misaligned
+ * tensors or a short workspace; VEDA_ERR_UNSUPPORTED for NT_max > 32767. */
+veda_status veda_tile_sparse_attn_backward_grid(const veda_problem* p, const void* q, const void* k, const void* v,
+                                                const void* o, const float* lse, const void* d_o,
+                                                const int32_t* idx, int32_t k_max, float scale, void* dq,
+                                                void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                                                void* stream);
+
 /* ---------------------------------------------------------------- status */
 
 /* Synchronises `stream`, then reads and clears the library's device error

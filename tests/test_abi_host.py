@@ -162,3 +162,30 @@ def test_head_error_validates_on_the_host(V):
     assert lib.veda_head_error(p.ref, None, 256, 256, 256, 256, 4096, None) == B.VEDA_ERR_INVALID_ARG
     assert lib.veda_head_error(p.ref, 8, 256, 256, 256, 256, 4096, None) == B.VEDA_ERR_INVALID_ARG
     assert lib.veda_head_error(p.ref, 256, 256, 256, 256, 256, 16, None) == B.VEDA_ERR_INVALID_ARG   # short workspace
+
+
+def test_attention_backward_validates_on_the_host(V):
+    """Workspace size from its parts; NULL, misaligned and short-workspace calls
+    are refused before any launch (pointers are never dereferenced)."""
+    B = V.binding
+    p = V.Problem(2, 3, 64, 64, (5, 13, 19), [(1, 8, 8), (4, 4, 4), (2, 4, 8)])
+    nt, k_max = p.nt_max, 5
+    r256 = lambda x: (x + 255) // 256 * 256
+    bh, N, W = 6, 5 * 13 * 19, (p.nt_max + 31) // 32
+    expect = r256(4 * bh * N) + r256(4 * bh * nt * W) + r256(4 * bh * (nt + 1)) + r256(4 * bh * nt * k_max)
+    assert V.veda_attn_backward_workspace(p, k_max) == expect
+    with pytest.raises(V.VedaError):
+        V.veda_attn_backward_workspace(p, 0)
+    lib = V.LIB
+    f = lib.veda_tile_sparse_attn_backward_grid
+    good = [256] * 7
+    args = lambda ptrs, k=k_max, sc=0.0, outs=(256, 256, 256), ws=4096, nb=1 << 30: (
+        p.ref, *ptrs, k, ctypes.c_float(sc), *outs, ws, nb, None)
+    assert f(*args([None] + good[1:])) == B.VEDA_ERR_INVALID_ARG                 # NULL q
+    assert f(*args(good[:4] + [None] + good[5:])) == B.VEDA_ERR_INVALID_ARG      # NULL lse
+    assert f(*args(good, outs=(256, 256, None))) == B.VEDA_ERR_INVALID_ARG      # NULL dv
+    assert f(*args(good[:5] + [8] + good[6:])) == B.VEDA_ERR_INVALID_ARG        # misaligned d_o
+    assert f(*args(good, ws=4096 + 16)) == B.VEDA_ERR_INVALID_ARG               # workspace not 256-aligned
+    assert f(*args(good, nb=expect - 1)) == B.VEDA_ERR_INVALID_ARG              # short workspace
+    assert f(*args(good, k=0)) == B.VEDA_ERR_INVALID_ARG
+    assert f(*args(good, sc=float("inf"))) == B.VEDA_ERR_INVALID_ARG

@@ -78,6 +78,9 @@ _SIG = {
                                _V, ctypes.POINTER(veda_mlp_grad), ctypes.POINTER(veda_mlp_grad), _V, ctypes.c_size_t,
                                _V],
     "veda_head_error": [_P, _V, _V, _V, _V, _V, ctypes.c_size_t, _V],
+    "veda_attn_backward_workspace": [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)],
+    "veda_tile_sparse_attn_backward_grid": [_P, _V, _V, _V, _V, _V, _V, _V, ctypes.c_int32, ctypes.c_float, _V, _V,
+                                            _V, _V, ctypes.c_size_t, _V],
     "veda_sync_status": [_V],
     "veda_set_wait_timeout_ns": [ctypes.c_uint64],
     "veda_selftest_wait_timeout": [ctypes.c_uint64, _V],
@@ -281,6 +284,29 @@ def veda_tile_sparse_attn_grid(p: Problem, q: torch.Tensor, k: torch.Tensor, v: 
         _ptr(lse, "lse", torch.float32, (p.B, p.heads, p.N)), _stream(stream)),
         "veda_tile_sparse_attn_grid")
     return o
+
+
+def veda_attn_backward_workspace(p: Problem, k_max: int) -> int:
+    n = ctypes.c_size_t()
+    _check(LIB.veda_attn_backward_workspace(p.ref, int(k_max), ctypes.byref(n)), "veda_attn_backward_workspace")
+    return int(n.value)
+
+
+def veda_tile_sparse_attn_backward_grid(p: Problem, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                        o: torch.Tensor, lse: torch.Tensor, d_o: torch.Tensor, idx: torch.Tensor,
+                                        dq: torch.Tensor, dk: torch.Tensor, dv: torch.Tensor,
+                                        workspace: torch.Tensor, scale: float = 0.0, stream=None):
+    """dq, dk, dv of veda_tile_sparse_attn_grid for the upstream gradient d_o (all grid order)."""
+    gs = p.grid_shape()
+    k_max = int(idx.shape[-1])
+    _check(LIB.veda_tile_sparse_attn_backward_grid(
+        p.ref, _ptr(q, "q", torch.bfloat16, gs), _ptr(k, "k", torch.bfloat16, gs), _ptr(v, "v", torch.bfloat16, gs),
+        _ptr(o, "o", torch.bfloat16, gs), _ptr(lse, "lse", torch.float32, (p.B, p.heads, p.N)),
+        _ptr(d_o, "d_o", torch.bfloat16, gs), _ptr(idx, "idx", torch.int32, (p.B, p.heads, p.nt_max, k_max)), k_max,
+        ctypes.c_float(scale), _ptr(dq, "dq", torch.bfloat16, gs), _ptr(dk, "dk", torch.bfloat16, gs),
+        _ptr(dv, "dv", torch.bfloat16, gs), _ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "veda_tile_sparse_attn_backward_grid")
+    return dq, dk, dv
 
 
 def veda_attn_config(p: Problem, k_max: int) -> Tuple[int, int, int]:

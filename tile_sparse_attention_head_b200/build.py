@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libveda.so")
 SOURCES = ["veda_api.cu", "veda_common.cuh", "kernels.h", "permute_tripool.cu", "score_topk.cu",
-           "sparse_attn.cu", "tile_map.cu", "estimator.cu", "distill.cu"]
+           "sparse_attn.cu", "tile_map.cu", "estimator.cu", "distill.cu", "attn_bwd.cu"]
 
 
 def nvcc_path() -> str:

@@ -48,6 +48,32 @@ struct AttnMaps {
   CUtensorMap q[NM], k[NM], v[NM];
 };
 
+// Attention backward (grid order).  The dQ launch holds (Q_i, dO_i) and
+// streams the selected (K, V) tiles; the dK/dV launch holds (K_j, V_j) and
+// streams (Q, dO) of the Q tiles that selected j.  Maps per distinct tiling:
+// a0/a1 the stationary pair, b0/b1 the moving pair.
+template <int NM>
+struct BwdMaps {
+  CUtensorMap a0[NM], a1[NM], b0[NM], b1[NM];
+};
+
+struct BwdArgs {
+  const int32_t* idx;       // [B, heads, NT_max, k_max]
+  int32_t k_max;
+  const int32_t* inv_off;   // [B*heads, NT_max + 1]
+  const int32_t* inv_list;  // [B*heads, NT_max * k_max]
+  const float* lse;         // [B, heads, N], natural log, scale included
+  const float* dsum;        // [B, heads, N], rowsum(dO * O)
+  void* dx;                 // bf16 [B, heads, N, d]: dQ (dQ launch) or dK (dK/dV launch)
+  void* dv;                 // bf16 [B, heads, N, d]: dV (dK/dV launch)
+  float scale;
+  float scale_log2;
+  uint64_t timeout_ns;
+  int32_t n_group;
+  int16_t head_list[VEDA_MAX_HEADS];
+  int8_t map_of_head[VEDA_MAX_HEADS];
+};
+
 struct MapArgs {
   const int32_t* rows;  // [B*heads, R]
   int32_t R;
@@ -93,6 +119,16 @@ cudaError_t launch_distill(const Geometry& G, const float* desc_q, const float* 
                            const EstimatorWeights& wk, int hidden, int e, const float* map, const int32_t* rows,
                            int R, float* loss, const EstimatorWeights& gq, const EstimatorWeights& gk, void* ws,
                            uint64_t timeout_ns, cudaStream_t s);
+
+size_t attn_bwd_ws_bytes(const Geometry& G, int k_max);
+size_t attn_bwd_smem_bytes(int d, int S);
+// D = rowsum(dO * O) and the inverse selection lists into the workspace; fills
+// a.idx, a.k_max, a.dsum, a.inv_off and a.inv_list.
+cudaError_t launch_attn_bwd_prep(const Geometry& G, const void* o, const void* dout, const int32_t* idx, int k_max,
+                                 void* ws, BwdArgs* a, cudaStream_t s);
+cudaError_t launch_attn_bwd_dq(const Geometry& G, const BwdMaps<kMaxGridMaps>& m, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_attn_bwd_dkdv(const Geometry& G, const BwdMaps<kMaxGridMaps>& m, const BwdArgs& a,
+                                 cudaStream_t s);
 
 cudaError_t launch_timeout_selftest(uint64_t timeout_ns, cudaStream_t s);
 

@@ -20,6 +20,7 @@
 #include "sparse_attn.cu"
 #include "tile_map.cu"
 #include "distill.cu"
+#include "attn_bwd.cu"
 
 namespace veda {
 namespace {
@@ -634,6 +635,95 @@ veda_status veda_head_error(const veda_problem* p, const void* o, const void* o_
   if (workspace_bytes < need) return fail(VEDA_ERR_INVALID_ARG, "workspace needs %zu bytes", need);
   cudaError_t ce = launch_head_error(G, o, o_ref, err, ref_sq, static_cast<float*>(workspace), (cudaStream_t)stream);
   if (ce != cudaSuccess) return cuda_fail(ce, "veda_head_error");
+  return ok();
+}
+
+veda_status veda_attn_backward_workspace(const veda_problem* p, int32_t k_max, size_t* bytes) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (k_max < 1) return fail(VEDA_ERR_INVALID_ARG, "k_max must be >= 1 (got %d)", k_max);
+  if (!bytes) return fail(VEDA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = attn_bwd_ws_bytes(G, k_max);
+  return ok();
+}
+
+veda_status veda_tile_sparse_attn_backward_grid(const veda_problem* p, const void* q, const void* k, const void* v,
+                                                const void* o, const float* lse, const void* d_o,
+                                                const int32_t* idx, int32_t k_max, float scale, void* dq,
+                                                void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                                                void* stream) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (!q || !k || !v || !o || !lse || !d_o || !idx || !dq || !dk || !dv || !workspace)
+    return fail(VEDA_ERR_INVALID_ARG, "NULL argument");
+  const void* ptrs[] = {q, k, v, o, lse, d_o, idx, dq, dk, dv};
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return fail(VEDA_ERR_INVALID_ARG, "tensor arguments must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(VEDA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (k_max < 1) return fail(VEDA_ERR_INVALID_ARG, "k_max must be >= 1 (got %d)", k_max);
+  if (!(std::isfinite(scale))) return fail(VEDA_ERR_INVALID_ARG, "scale must be finite");
+  if (G.ntmax > 32767) return fail(VEDA_ERR_UNSUPPORTED, "NT_max = %d exceeds 32767 tiles per head", G.ntmax);
+  if (workspace_bytes < attn_bwd_ws_bytes(G, k_max))
+    return fail(VEDA_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu required", workspace_bytes,
+                attn_bwd_ws_bytes(G, k_max));
+  const cudaStream_t st = (cudaStream_t)stream;
+  BwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  cudaError_t ce = launch_attn_bwd_prep(G, o, d_o, idx, k_max, workspace, &a, st);
+  if (ce != cudaSuccess) return cuda_fail(ce, "veda_tile_sparse_attn_backward_grid (prep)");
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)G.d);
+  a.scale = sc;
+  a.scale_log2 = sc * 1.4426950408889634f;
+  a.lse = lse;
+  a.timeout_ns = g_timeout_ns;
+  // Distinct tilings in order of first appearance, up to kMaxGridMaps per launch.
+  int tiling_of_head[VEDA_MAX_HEADS];
+  int distinct[VEDA_MAX_HEADS];
+  int n_distinct = 0;
+  for (int h = 0; h < G.heads; ++h) {
+    int u = 0;
+    while (u < n_distinct && !(G.g[distinct[u]].pt == G.g[h].pt && G.g[distinct[u]].ph == G.g[h].ph &&
+                               G.g[distinct[u]].pw == G.g[h].pw))
+      ++u;
+    if (u == n_distinct) distinct[n_distinct++] = h;
+    tiling_of_head[h] = u;
+  }
+  BwdMaps<kMaxGridMaps> mq, mkv;   // copied into the kernel parameters at launch
+  std::memset(&mq, 0, sizeof(mq));
+  std::memset(&mkv, 0, sizeof(mkv));
+  for (int u0 = 0; u0 < n_distinct; u0 += kMaxGridMaps) {
+    const int nu = std::min(kMaxGridMaps, n_distinct - u0);
+    for (int u = 0; u < nu; ++u) {
+      const HeadGeom& hg = G.g[distinct[u0 + u]];
+      if ((s = encode_grid_tiles(G, q, hg, &mq.a0[u])) != VEDA_OK ||
+          (s = encode_grid_tiles(G, d_o, hg, &mq.a1[u])) != VEDA_OK ||
+          (s = encode_grid_tiles(G, k, hg, &mq.b0[u])) != VEDA_OK ||
+          (s = encode_grid_tiles(G, v, hg, &mq.b1[u])) != VEDA_OK)
+        return s;
+      mkv.a0[u] = mq.b0[u];   // K
+      mkv.a1[u] = mq.b1[u];   // V
+      mkv.b0[u] = mq.a0[u];   // Q
+      mkv.b1[u] = mq.a1[u];   // dO
+    }
+    a.n_group = 0;
+    for (int h = 0; h < G.heads; ++h) {
+      const int u = tiling_of_head[h] - u0;
+      if (u < 0 || u >= nu) continue;
+      a.head_list[a.n_group++] = (int16_t)h;
+      a.map_of_head[h] = (int8_t)u;
+    }
+    a.dx = dq;
+    a.dv = nullptr;
+    if ((ce = launch_attn_bwd_dq(G, mq, a, st)) != cudaSuccess)
+      return cuda_fail(ce, "veda_tile_sparse_attn_backward_grid (dQ)");
+    a.dx = dk;
+    a.dv = dv;
+    if ((ce = launch_attn_bwd_dkdv(G, mkv, a, st)) != cudaSuccess)
+      return cuda_fail(ce, "veda_tile_sparse_attn_backward_grid (dK, dV)");
+  }
   return ok();
 }
 

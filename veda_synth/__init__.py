@@ -147,6 +147,18 @@ def make_qkv(w: Workload, seed: int = 0, heads: Optional[int] = None):
             torch.stack(vs, 1).contiguous())
 
 
+def make_grad_out(w: Workload, seed: int = 4, heads: Optional[int] = None) -> torch.Tensor:
+    """An upstream gradient dO for the attention backward: bf16 CPU tensor
+    [B, heads, N, d] in grid order, N(0,1) drawn in fp32 per head from its own
+    sub-seed and rounded to bf16."""
+    H_ = w.heads if heads is None else heads
+    outs = []
+    for h in range(H_):
+        g = torch.Generator().manual_seed(seed * 100019 + h)
+        outs.append(torch.randn((w.B, w.N, w.d), generator=g).to(torch.bfloat16))
+    return torch.stack(outs, 1).contiguous()
+
+
 @dataclass
 class MLPWeights:
     """Per-head two-layer estimator weights, fp32: W1 [heads,hid,3d], b1 [heads,hid], W2 [heads,e,hid], b2 [heads,e]."""
