@@ -314,6 +314,41 @@ def attention_sustained(V, p, att, qd, kd, vd, out, args, flops, local):
     return {"launches": n, "ms_per_launch": ms, "tflops": flops / (ms * 1e-3) / 1e12, "clocks": clk}
 
 
+def backward_measure(V, w, p, att, qd, kd, vd, args, flops, rank, dev):
+    """The attention backward (dQ, dK, dV over the selected tiles) after the
+    layer's forward, timed over args.bwd_steps calls with CUDA events.  Its
+    algorithmic work is the usual 2.5x the forward's kept-tile FLOPs (five
+    S x S x d products per kept pair: S, dP, dV, dQ, dK); the kernels run
+    seven (S and dP once for dQ and once for dK/dV)."""
+    from veda_synth import make_grad_out
+    if args.layout != "grid":
+        return {"skipped": "the backward runs on grid-order tensors (--layout grid)"}
+    o = torch.empty(p.grid_shape(), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((p.B, p.heads, p.N), dtype=torch.float32, device=dev)
+    V.veda_tile_sparse_attn_grid(p, qd, kd, vd, att.idx, o, lse)
+    do = make_grad_out(w, seed=rank + 4).to(dev)
+    grads = [torch.empty_like(qd) for _ in range(3)]
+    ws = torch.empty(V.veda_attn_backward_workspace(p, int(att.idx.shape[-1])), dtype=torch.uint8, device=dev)
+    step = lambda: V.veda_tile_sparse_attn_backward_grid(p, qd, kd, vd, o, lse, do, att.idx, *grads, ws)
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.bwd_steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    V.veda_sync_status()
+    ms = e0.elapsed_time(e1) / args.bwd_steps
+    peaks, src = load_peaks()
+    alg = 2.5 * flops / (ms * 1e-3) / 1e12
+    return {"ms": ms, "algorithmic_flops": 2.5 * flops, "tflops": alg,
+            "executed_tflops": 3.5 * flops / (ms * 1e-3) / 1e12,
+            "frac_of_sustained_peak": alg / peaks["bf16_tflops_sustained"], "peak_source": src,
+            "ratio_to_forward_attention": None}
+
+
 def run_ours(args, world, rank, local):
     import tile_sparse_attention_head_b200 as V
     from veda_synth import PRESETS, make_mlp, make_qkv
@@ -432,6 +467,9 @@ def run_ours(args, world, rank, local):
         sustained = attention_sustained(V, p, att, qd, kd, vd, out, args, flops, local)
     useful = useful_flops(w, att.idx.cpu().numpy())
     tmap = tile_map_measure(V, w, p, qd, kd, args, rank, att) if args.map else None
+    bwd = backward_measure(V, w, p, att, qd, kd, vd, args, flops, rank, dev) if args.bwd else None
+    if bwd is not None and "ms" in bwd:
+        bwd["ratio_to_forward_attention"] = bwd["ms"] / attn_ms
     res = {"metric": METRIC, "value": weak_scaling_value(flops, ms_step, world), "unit": "TFLOP/s",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -444,6 +482,8 @@ def run_ours(args, world, rank, local):
         res["attention_sustained"] = sustained
     if tmap is not None:
         res["tile_map"] = tmap
+    if bwd is not None:
+        res["backward"] = bwd
     return res, (w, p, ks, flops)
 
 
@@ -518,6 +558,8 @@ def main():
                     help="keep ratio k / NT_max, i.e. k selected tiles per Q tile (the fixed-k token sweep)")
     ap.add_argument("--map", action="store_true", help="also time the max-pooled tile map (10%% of Q tiles)")
     ap.add_argument("--map-steps", type=int, default=5)
+    ap.add_argument("--bwd", action="store_true", help="also time the attention backward (dQ, dK, dV)")
+    ap.add_argument("--bwd-steps", type=int, default=5)
     ap.add_argument("--attn-sustain", type=float, default=0.0,
                     help="also run the attention kernel back to back for this many seconds, sampling clock and power")
     ap.add_argument("--no-cpu-baseline", action="store_true")

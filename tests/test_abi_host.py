@@ -172,7 +172,7 @@ def test_attention_backward_validates_on_the_host(V):
     nt, k_max = p.nt_max, 5
     r256 = lambda x: (x + 255) // 256 * 256
     bh, N, W = 6, 5 * 13 * 19, (p.nt_max + 31) // 32
-    expect = r256(4 * bh * N) + r256(4 * bh * nt * W) + r256(4 * bh * (nt + 1)) + r256(4 * bh * nt * k_max)
+    expect = r256(8 * bh * nt * 64) + r256(4 * bh * nt * W) + r256(4 * bh * (nt + 1)) + r256(4 * bh * nt * k_max)
     assert V.veda_attn_backward_workspace(p, k_max) == expect
     with pytest.raises(V.VedaError):
         V.veda_attn_backward_workspace(p, 0)

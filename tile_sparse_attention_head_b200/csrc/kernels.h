@@ -62,8 +62,8 @@ struct BwdArgs {
   int32_t k_max;
   const int32_t* inv_off;   // [B*heads, NT_max + 1]
   const int32_t* inv_list;  // [B*heads, NT_max * k_max]
-  const float* lse;         // [B, heads, N], natural log, scale included
-  const float* dsum;        // [B, heads, N], rowsum(dO * O)
+  const float2* ldt;        // [B*heads, NT_max, S]: per tile slot (L, D) = (lse log2(e), rowsum(dO * O)),
+                            // (+inf, 0) on pad slots
   void* dx;                 // bf16 [B, heads, N, d]: dQ (dQ launch) or dK (dK/dV launch)
   void* dv;                 // bf16 [B, heads, N, d]: dV (dK/dV launch)
   float scale;
@@ -121,11 +121,10 @@ cudaError_t launch_distill(const Geometry& G, const float* desc_q, const float* 
                            uint64_t timeout_ns, cudaStream_t s);
 
 size_t attn_bwd_ws_bytes(const Geometry& G, int k_max);
-size_t attn_bwd_smem_bytes(int d, int S);
-// D = rowsum(dO * O) and the inverse selection lists into the workspace; fills
-// a.idx, a.k_max, a.dsum, a.inv_off and a.inv_list.
-cudaError_t launch_attn_bwd_prep(const Geometry& G, const void* o, const void* dout, const int32_t* idx, int k_max,
-                                 void* ws, BwdArgs* a, cudaStream_t s);
+// Per tile slot (L, D) and the inverse selection lists into the workspace;
+// fills a.idx, a.k_max, a.ldt, a.inv_off and a.inv_list.
+cudaError_t launch_attn_bwd_prep(const Geometry& G, const void* o, const void* dout, const float* lse,
+                                 const int32_t* idx, int k_max, void* ws, BwdArgs* a, cudaStream_t s);
 cudaError_t launch_attn_bwd_dq(const Geometry& G, const BwdMaps<kMaxGridMaps>& m, const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_attn_bwd_dkdv(const Geometry& G, const BwdMaps<kMaxGridMaps>& m, const BwdArgs& a,
                                  cudaStream_t s);

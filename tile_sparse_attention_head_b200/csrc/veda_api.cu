@@ -672,12 +672,11 @@ veda_status veda_tile_sparse_attn_backward_grid(const veda_problem* p, const voi
   const cudaStream_t st = (cudaStream_t)stream;
   BwdArgs a;
   std::memset(&a, 0, sizeof(a));
-  cudaError_t ce = launch_attn_bwd_prep(G, o, d_o, idx, k_max, workspace, &a, st);
+  cudaError_t ce = launch_attn_bwd_prep(G, o, d_o, lse, idx, k_max, workspace, &a, st);
   if (ce != cudaSuccess) return cuda_fail(ce, "veda_tile_sparse_attn_backward_grid (prep)");
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)G.d);
   a.scale = sc;
   a.scale_log2 = sc * 1.4426950408889634f;
-  a.lse = lse;
   a.timeout_ns = g_timeout_ns;
   // Distinct tilings in order of first appearance, up to kMaxGridMaps per launch.
   int tiling_of_head[VEDA_MAX_HEADS];
