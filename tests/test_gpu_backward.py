@@ -124,3 +124,81 @@ def test_backward_unselected_keys_get_zero_and_is_deterministic(V):
     for name, g, ref in zip(("dq", "dk", "dv"), g1, refs):
         for h in range(2):
             check_grad(name, f64(g[0, h]), ref[0, h], f"one tile h{h}")
+
+
+def _oracle_dkdv_tile(qp, kp, vp, dop, tab, idx_rows, j, S, scale):
+    """dK, dV rows (slot order) of K tile j of one head: the sum over every Q
+    tile whose selection holds j of its contribution to j's keys."""
+    d = qp.shape[1]
+    dk, dv = np.zeros((S, d)), np.zeros((S, d))
+    for i, row in enumerate(idx_rows):
+        sel = row[row >= 0]
+        if j not in sel:
+            continue
+        _, kr, dki, dvi = O.attention_tile_backward(qp, kp, vp, dop, tab, i, sel, S, scale)
+        m = (kr // S) == j
+        dk[kr[m] % S] += dki[m]
+        dv[kr[m] % S] += dvi[m]
+    return dk, dv
+
+
+def test_backward_wan14b_full_size_sampled(V):
+    """The benchmarked 14B shape (40 heads, grid order, the launch the bench
+    times): dQ of sampled Q tiles and dK, dV of sampled K tiles (the most
+    selected one and random ones) of two heads against the oracle, with the
+    oracle's selection for those heads."""
+    w = PRESETS["wan14b"]
+    p = _problem(V, w)
+    grid = (w.T, w.H, w.W)
+    q, k, v = make_qkv(w, seed=0)
+    do = make_grad_out(w, seed=4)
+    m = make_mlp(w, seed=1)
+    md = tuple(t.cuda() for t in (m.w1, m.b1, m.w2, m.b2))
+    att = V.VedaAttention(p, md, md, w.keep, layout="grid")
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    att(qd, kd, vd)
+    V.veda_sync_status()
+    idx = att.idx.clone()
+    k_max = idx.shape[-1]
+    mlp_all = mlp_numpy(m)
+    heads = (5, 30)
+    ora = {}
+    for h in heads:
+        tl = [w.tilings[h]]
+        mh = tuple(a[h:h + 1] for a in mlp_all)
+        qp, kp, vp, dop = (O.tile_permute(f64(t[:, h:h + 1]), grid, tl, w.S) for t in (q, k, v, do))
+        dq_, dk_ = O.tripool(qp, grid, tl, w.S), O.tripool(kp, grid, tl, w.S)
+        oi = O.score_topk(dq_, dk_, grid, tl, w.S, mh, mh, keep_f32(w.keep))[0][0, 0]
+        nt = p.nt_per_head[h]
+        row = np.full((p.nt_max, k_max), -1, dtype=np.int32)
+        row[:nt, :oi.shape[1]] = oi[:nt]
+        idx[0, h] = torch.from_numpy(row).cuda()
+        ora[h] = (qp[0, 0], kp[0, 0], vp[0, 0], dop[0, 0], row[:nt])
+    grads = gpu_backward(V, p, qd, kd, vd, dod, idx)
+    rng = np.random.default_rng(3)
+    scale = 1 / np.sqrt(w.d)
+    checked = 0
+    for h in heads:
+        qp, kp, vp, dop, rows = ora[h]
+        tab = O.slot_table(grid, w.tilings[h])
+        nt = rows.shape[0]
+        for i in rng.choice(nt, 3, replace=False):
+            dq_ref, _, _, _ = O.attention_tile_backward(qp, kp, vp, dop, tab, int(i), rows[i][rows[i] >= 0], w.S, scale)
+            slots = np.nonzero(tab[i * w.S:(i + 1) * w.S] >= 0)[0]
+            n = torch.from_numpy(tab[i * w.S:(i + 1) * w.S][slots]).cuda()
+            check_grad("dq", f64(grads[0][0, h, n]), dq_ref[slots], f"h{h} Q tile {i}")
+            checked += 1
+        counts = np.bincount(rows[rows >= 0], minlength=nt)
+        for j in [int(np.argmax(counts))] + [int(x) for x in rng.choice(nt, 2, replace=False)]:
+            dk_ref, dv_ref = _oracle_dkdv_tile(qp, kp, vp, dop, tab, rows, j, w.S, scale)
+            slots = np.nonzero(tab[j * w.S:(j + 1) * w.S] >= 0)[0]
+            n = torch.from_numpy(tab[j * w.S:(j + 1) * w.S][slots]).cuda()
+            if counts[j] == 0:
+                assert torch.count_nonzero(grads[1][0, h, n]) == 0 and torch.count_nonzero(grads[2][0, h, n]) == 0
+                continue
+            check_grad("dk", f64(grads[1][0, h, n]), dk_ref[slots], f"h{h} K tile {j} ({counts[j]} selections)")
+            check_grad("dv", f64(grads[2][0, h, n]), dv_ref[slots], f"h{h} K tile {j}")
+            checked += 1
+    assert checked >= 10
+    for g in grads:
+        assert bool(torch.isfinite(g.float()).all())
