@@ -13,7 +13,10 @@
  *
  *   veda_tripool_grid (Q, K)  ->  veda_tile_score_topk  ->  veda_tile_sparse_attn_grid
  *
- * and the distillation target is built by veda_tile_map_maxpool.
+ * and the distillation target is built by veda_tile_map_maxpool.  Training
+ * calls: veda_distill_loss_grad (the estimator's row-wise KL loss and MLP
+ * gradients) and veda_tile_sparse_attn_backward_grid (dQ, dK, dV of the
+ * grid-order attention over the same selected tiles).
  *
  * Conventions shared by every call
  * --------------------------------
