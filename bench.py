@@ -580,8 +580,8 @@ def main():
     res, (w, p, ks, flops) = run_ours(args, world, rank, local)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            # bounded sample: 3 whole heads (~10 s of CPU work on the bench host)
-            secs, done, desc = cpu_sample_oracle(w, p.nt_per_head, ks, heads=min(3, w.heads), tiles=None)
+            # bounded sample: 5 whole heads (~12-15 s of CPU work on the bench host)
+            secs, done, desc = cpu_sample_oracle(w, p.nt_per_head, ks, heads=min(5, w.heads), tiles=None)
             res["cpu_baseline"] = {"value": done / secs / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
                                    "kind": "oracle", "sample": desc, "seconds": secs}
         print(json.dumps(res), flush=True)
