@@ -8,9 +8,14 @@
 //                     on the tensor cores at fp32 accuracy (estimator.cu),
 //                     written to the workspace;
 //   score_topk_kernel per block of Q-tile rows: s = phi_q phi_k^T / sqrt(e)
-//                     into shared memory, optional row softmax, then an exact
-//                     radix select of the k-th largest score per row and an
-//                     ascending compaction of the winners.
+//                     into shared memory, optional row softmax, then the
+//                     exact k-th largest score per row and an ascending
+//                     compaction of the winners.  Rows of up to 2048 tiles
+//                     find the k-th largest by bisection over order-preserving
+//                     32-bit keys held in registers (one warp per row, a
+//                     compare-and-count per step, no shared-memory traffic);
+//                     longer rows use a 4-pass radix select over shared
+//                     histograms.
 // Scores stay fp32 end to end so that selections only differ from an exact
 // evaluation on genuine near-ties.
 #include "veda_common.cuh"
@@ -25,6 +30,54 @@ __device__ __forceinline__ uint32_t float_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// k-th largest key of a row by bisection: each lane holds keys of columns
+// lane, lane + 32, ... (KPL of them, 0 past the row end; every real key is
+// above 0).  Returns the key value t and, in *gt, the number of keys above t.
+// Invariant: count(key >= lo) >= k > count(key >= hi); a midpoint with exactly
+// k keys at or above it ends the search early.
+template <int KPL>
+__device__ __forceinline__ uint32_t kth_key_bisect(const uint32_t (&key)[KPL], int nt, int k, int lane, int* gt) {
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i)
+    if (i * 32 + lane < nt) {
+      kmin = min(kmin, key[i]);
+      kmax = max(kmax, key[i]);
+    }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  auto count_ge = [&](uint32_t t) {
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) c += key[i] >= t ? 1 : 0;
+    return (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+  };
+  uint64_t lo = kmin, hi = (uint64_t)kmax + 1;
+  uint32_t t = 0;
+  bool found = false;
+  while (hi - lo > 1) {
+    const uint64_t mid = lo + ((hi - lo) >> 1);
+    const int c = count_ge((uint32_t)mid);
+    if (c == k) {   // exactly the k largest are >= mid: t is the smallest of them
+      uint32_t m = 0xffffffffu;
+#pragma unroll
+      for (int i = 0; i < KPL; ++i)
+        if (key[i] >= (uint32_t)mid) m = min(m, key[i]);
+      t = __reduce_min_sync(0xffffffffu, m);
+      found = true;
+      break;
+    }
+    if (c > k) lo = mid;
+    else hi = mid;
+  }
+  if (!found) t = (uint32_t)lo;
+  int c = 0;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) c += key[i] > t ? 1 : 0;
+  *gt = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+  return t;
+}
+
 constexpr int kScoreThreads = 256;
 constexpr int kKChunk = 128;       // K tiles staged per step
 constexpr int kQRows = 16;         // most Q-tile rows per CTA (the score tile is 16 x 128)
@@ -34,6 +87,7 @@ constexpr int kQRows = 16;         // most Q-tile rows per CTA (the score tile i
 // a score step is one float2 and one float4 load feeding 8 FMAs: thread t
 // forms rows 2(t/32), 2(t/32)+1 x columns 4(t%32)..+3 of the 16 x 128 tile),
 // radix histograms [8][256].
+template <int KPL>
 __global__ void __launch_bounds__(kScoreThreads)
     score_topk_kernel(const __grid_constant__ Geometry G, const float* __restrict__ phi, int e,
                       int qb, int ntpad, const __grid_constant__ TopkArgs args) {
@@ -143,9 +197,22 @@ __global__ void __launch_bounds__(kScoreThreads)
       for (int c = lane; c < G.ntmax; c += 32) prow[c] = (c < nt) ? expf(srow[c] - m) * inv : 0.f;
     }
 
-    // Radix select: find the k-th largest key, 8 bits per pass from the top.
-    uint32_t prefix = 0, pmask = 0;
+    uint32_t prefix = 0;
     int remaining = k;
+    if (KPL > 0 && nt <= 32 * KPL) {
+      // Bisection over the keys, held in registers.
+      uint32_t key[KPL > 0 ? KPL : 1];
+#pragma unroll
+      for (int i = 0; i < (KPL > 0 ? KPL : 1); ++i) {
+        const int c = i * 32 + lane;
+        key[i] = c < nt ? float_key(srow[c]) : 0u;
+      }
+      int gt = 0;
+      prefix = kth_key_bisect(key, nt, k, lane, &gt);
+      remaining = k - gt;
+    } else {
+    // Radix select: find the k-th largest key, 8 bits per pass from the top.
+    uint32_t pmask = 0;
 #pragma unroll 1
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int b = lane; b < 256; b += 32) hist[b] = 0;
@@ -193,6 +260,7 @@ __global__ void __launch_bounds__(kScoreThreads)
       pmask |= 255u << shift;
       __syncwarp();
     }
+    }
     // prefix = k-th largest key; take every key above it and the first
     // `remaining` keys equal to it (smallest tile indices), in ascending order.
     int out = 0, eq_taken = 0;
@@ -225,11 +293,17 @@ cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const floa
   int qb, ntpad;
   size_t smem;
   score_topk_config(G.ntmax, e, &qb, &ntpad, &smem);
-  err = cudaFuncSetAttribute(score_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (err != cudaSuccess) return err;
   dim3 g2((G.ntmax + qb - 1) / qb, G.B * G.heads);
-  score_topk_kernel<<<g2, kScoreThreads, smem, s>>>(G, phi, e, qb, ntpad, args);
-  return cudaGetLastError();
+  // keys per lane of the register bisection: the row length it covers is 32 x KPL
+  auto go = [&](auto kernel) -> cudaError_t {
+    cudaError_t e2 = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e2 != cudaSuccess) return e2;
+    kernel<<<g2, kScoreThreads, smem, s>>>(G, phi, e, qb, ntpad, args);
+    return cudaGetLastError();
+  };
+  if (G.ntmax <= 32 * 32) return go(score_topk_kernel<32>);
+  if (G.ntmax <= 32 * 64) return go(score_topk_kernel<64>);
+  return go(score_topk_kernel<0>);
 }
 
 // Rows per CTA so that the score block fits in ~160 KB of shared memory.
