@@ -384,24 +384,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x on the FMA/ALU pipes, to take part of the exponential load off the
-// special-function unit.  x = j + f with j = round(x) and f in [-1/2, 1/2]
-// (rounding by adding and subtracting 1.5*2^23); 2^f is a cubic whose
-// coefficients were fitted for this library by a Remez exchange on the
-// relative error over [-1/2, 1/2] (max relative error 7.5e-5, far below the
-// bf16 rounding the attention probabilities get next); j is added to the
-// exponent field.  Inputs below -126 (including -inf) are clamped to -126,
-// i.e. give 2^-126 instead of 0.  Valid up to x = 127.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  float p = fmaf(0.0551716685f, f, 0.2426111251f);
-  p = fmaf(p, f, 0.6932609677f);
-  p = fmaf(p, f, 0.9999280572f);
-  return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
-}
-
 // Packed two-lane fp32 arithmetic (sm_100: fma/add.rn.f32x2 on a register pair).
 __device__ __forceinline__ uint64_t f2(float lo, float hi) {
   uint64_t r;
@@ -432,10 +414,18 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// exp2_fma on a pair of lanes: the reduction and the cubic run as packed
-// f32x2 operations, the exponent insertion per lane.  With t = x + 1.5*2^23
-// the bits of t are 0x4B400000 + j, and 0x4B400000 << 23 vanishes modulo
-// 2^32, so adding bits(t) << 23 to the cubic's bits adds j to its exponent.
+// 2^x for a pair of lanes on the FMA/ALU pipes, to take part of the
+// exponential load off the special-function unit.  x = j + f with
+// j = round(x) and f in [-1/2, 1/2] (rounding by adding and subtracting
+// 1.5*2^23); 2^f is a cubic whose coefficients were fitted for this library
+// by a Remez exchange on the relative error over [-1/2, 1/2] (max relative
+// error 7.5e-5, far below the bf16 rounding the probabilities get next); j is
+// added to the exponent field.  Inputs below -126 (including -inf) are
+// clamped to -126, i.e. give 2^-126 instead of 0.  Valid up to x = 127.
+// The reduction and the cubic run as packed f32x2 operations, the exponent
+// insertion per lane: with t = x + 1.5*2^23 the bits of t are 0x4B400000 + j,
+// and 0x4B400000 << 23 vanishes modulo 2^32, so adding bits(t) << 23 to the
+// cubic's bits adds j to its exponent.
 __device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& y0, float& y1) {
   const uint64_t x = f2(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
   const uint64_t magic = f2(12582912.0f, 12582912.0f);
