@@ -202,3 +202,23 @@ def test_backward_wan14b_full_size_sampled(V):
     assert checked >= 10
     for g in grads:
         assert bool(torch.isfinite(g.float()).all())
+
+
+def test_autograd_op_equals_the_c_abi_calls(V):
+    """tile_sparse_attention (torch autograd) gives exactly the output and the
+    gradients of the direct calls; VedaAttention.differentiable selects first."""
+    w = SMALL[2]                                       # odd128: B = 2, 4 heads, ragged tiles
+    p = _problem(V, w)
+    q, k, v = (t.cuda() for t in make_qkv(w, seed=6))
+    do = make_grad_out(w, seed=7).cuda()
+    md = tuple(t.cuda() for t in (lambda m: (m.w1, m.b1, m.w2, m.b2))(make_mlp(w, seed=1)))
+    att = V.VedaAttention(p, md, md, w.keep, layout="grid")
+    qa, ka, va = (t.clone().requires_grad_(True) for t in (q, k, v))
+    o = att.differentiable(qa, ka, va)
+    o.backward(do)
+    V.veda_sync_status()
+    ref = gpu_backward(V, p, q, k, v, do, att.idx)
+    o_ref = att(q, k, v)
+    assert torch.equal(o.detach(), o_ref)
+    for t, r in zip((qa, ka, va), ref):
+        assert torch.equal(t.grad, r)

@@ -11,5 +11,5 @@ from .binding import (  # noqa: F401
     veda_set_wait_timeout_ns, veda_sync_status, veda_tile_map_maxpool, veda_tile_map_workspace, veda_tile_permute, veda_tile_permute_tripool,
     veda_tile_score_topk, veda_tile_sparse_attn, veda_tile_sparse_attn_backward_grid, veda_tile_sparse_attn_grid, veda_tile_unpermute, veda_tripool,
     veda_tripool_grid, veda_version)
-from .pipeline import VedaAttention, VedaAttentionHost  # noqa: F401
+from .pipeline import VedaAttention, VedaAttentionHost, tile_sparse_attention  # noqa: F401
 from .tiling_search import tiling_search  # noqa: F401

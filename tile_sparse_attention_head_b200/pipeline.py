@@ -15,6 +15,12 @@ tile as a box of the grid-order tensor and writes grid rows)
 which is the per-layer path of Veda's tile-sparse attention (technical
 summary, sections 2.1-2.3).  Every step runs in the library's kernels; both
 layouts give the same output.
+
+``tile_sparse_attention`` is the grid-order attention as a differentiable
+torch op for a given selection: its forward is veda_tile_sparse_attn_grid
+(with the LSE kept for later), its backward veda_tile_sparse_attn_backward_grid.
+``VedaAttention.differentiable`` selects (without gradient: top-k is
+piecewise constant) and applies it.
 """
 from __future__ import annotations
 
@@ -23,6 +29,39 @@ from typing import Optional
 import torch
 
 from . import binding as B
+
+
+class _TileSparseAttention(torch.autograd.Function):
+    """Grid-order tile-skipping attention over a fixed selection, with the
+    library's backward; torch only holds the saved tensors."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, problem, idx):
+        p = problem
+        o = torch.empty(p.grid_shape(), dtype=torch.bfloat16, device=q.device)
+        lse = torch.empty((p.B, p.heads, p.N), dtype=torch.float32, device=q.device)
+        B.veda_tile_sparse_attn_grid(p, q, k, v, idx, o, lse)
+        ctx.problem = p
+        ctx.save_for_backward(q, k, v, o, lse, idx)
+        return o
+
+    @staticmethod
+    def backward(ctx, d_o):
+        q, k, v, o, lse, idx = ctx.saved_tensors
+        p = ctx.problem
+        d_o = d_o.to(torch.bfloat16).contiguous()
+        dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+        ws = torch.empty(B.veda_attn_backward_workspace(p, int(idx.shape[-1])), dtype=torch.uint8, device=q.device)
+        B.veda_tile_sparse_attn_backward_grid(p, q, k, v, o, lse, d_o, idx, dq, dk, dv, ws)
+        return dq, dk, dv, None, None
+
+
+def tile_sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, problem: B.Problem,
+                          idx: torch.Tensor) -> torch.Tensor:
+    """Differentiable tile-skipping attention: grid-order bf16 q, k, v
+    [B, heads, N, d] attend over the K tiles listed in idx
+    [B, heads, NT_max, k_max] (scale 1/sqrt(d)); gradients flow to q, k and v."""
+    return _TileSparseAttention.apply(q, k, v, problem, idx)
 
 
 class VedaAttention:
@@ -91,6 +130,15 @@ class VedaAttention:
             B.veda_tile_sparse_attn_grid(p, q, k, v, self.idx, out, self.lse, 0.0, stream)
         return out
 
+
+    def differentiable(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> torch.Tensor:
+        """Select tiles (no gradient), then the differentiable grid-order
+        attention over that selection (layout "grid" only)."""
+        if self.layout != "grid":
+            raise ValueError("the differentiable path runs on grid-order tensors (layout='grid')")
+        with torch.no_grad():
+            idx = self.select(q.detach(), k.detach(), v.detach()).clone()
+        return tile_sparse_attention(q, k, v, self.p, idx)
 
 class VedaAttentionHost:
     """The layer on HOST buffers: pinned grid-order bf16 Q, K, V in, O out.
