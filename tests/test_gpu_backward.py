@@ -222,3 +222,22 @@ def test_autograd_op_equals_the_c_abi_calls(V):
     assert torch.equal(o.detach(), o_ref)
     for t, r in zip((qa, ka, va), ref):
         assert torch.equal(t.grad, r)
+
+
+def test_backward_invalid_idx_entries_end_the_list(V):
+    """An entry outside [0, NT_h) ends a selection list like -1 does, for the
+    dQ side (the row's prefix) and the dK/dV side (the inverse lists) alike."""
+    w = SMALL[2]
+    p = _problem(V, w)
+    q, k, v = (t.cuda() for t in make_qkv(w, seed=3))
+    do = make_grad_out(w, seed=8).cuda()
+    idx = torch.full((p.B, p.heads, p.nt_max, 4), -1, dtype=torch.int32)
+    idx[..., 0] = 0
+    idx[..., 1] = 1
+    idx2 = idx.clone()
+    idx2[..., 2] = 10_000           # out of range: ends the list
+    idx2[..., 3] = 2
+    g1 = gpu_backward(V, p, q, k, v, do, idx.cuda())
+    g2 = gpu_backward(V, p, q, k, v, do, idx2.cuda())
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
