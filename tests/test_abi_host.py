@@ -189,3 +189,16 @@ def test_attention_backward_validates_on_the_host(V):
     assert f(*args(good, nb=expect - 1)) == B.VEDA_ERR_INVALID_ARG              # short workspace
     assert f(*args(good, k=0)) == B.VEDA_ERR_INVALID_ARG
     assert f(*args(good, sc=float("inf"))) == B.VEDA_ERR_INVALID_ARG
+
+
+def test_differentiable_path_requires_the_grid_layout(V):
+    """The autograd path runs on grid-order tensors; a tile-major layer refuses
+    it on the host before anything is launched (buffers here live on the CPU)."""
+    import torch
+    p = V.Problem(1, 1, 64, 64, (4, 8, 8), [(1, 8, 8)])
+    hid, e = 128, 32
+    mlp = (torch.zeros(1, hid, 192), torch.zeros(1, hid), torch.zeros(1, e, hid), torch.zeros(1, e))
+    att = V.VedaAttention(p, mlp, mlp, 0.5, device="cpu", layout="tile")
+    q = torch.zeros(p.grid_shape(), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        att.differentiable(q, q, q)
