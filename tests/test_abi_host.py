@@ -191,14 +191,14 @@ def test_attention_backward_validates_on_the_host(V):
     assert f(*args(good, sc=float("inf"))) == B.VEDA_ERR_INVALID_ARG
 
 
-def test_differentiable_path_requires_the_grid_layout(V):
-    """The autograd path runs on grid-order tensors; a tile-major layer refuses
-    it on the host before anything is launched (buffers here live on the CPU)."""
+def test_host_tensors_are_refused_no_cpu_fallback(V):
+    """The binding accepts device tensors only: a layer built on host memory
+    fails loudly at construction instead of falling back to a CPU path."""
     import torch
     p = V.Problem(1, 1, 64, 64, (4, 8, 8), [(1, 8, 8)])
     hid, e = 128, 32
     mlp = (torch.zeros(1, hid, 192), torch.zeros(1, hid), torch.zeros(1, e, hid), torch.zeros(1, e))
-    att = V.VedaAttention(p, mlp, mlp, 0.5, device="cpu", layout="tile")
-    q = torch.zeros(p.grid_shape(), dtype=torch.bfloat16)
-    with pytest.raises(ValueError):
-        att.differentiable(q, q, q)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        V.VedaAttention(p, mlp, mlp, 0.5, device="cpu", layout="tile")
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        V.make_mlp(*mlp)
