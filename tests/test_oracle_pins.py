@@ -246,6 +246,69 @@ def test_score_topk_contract():
             np.testing.assert_allclose(probs[0, h, i, :nt].sum(), 1.0, rtol=1e-13)
 
 
+def _mlp_by_loops(x, w1, b1, w2, b2):
+    """phi = W2 relu(W1 x + b1) + b2 for one descriptor row, written out as plain loops."""
+    hidden = []
+    for u in range(len(b1)):
+        z = b1[u]
+        for c in range(len(x)):
+            z += w1[u][c] * x[c]
+        hidden.append(z if z > 0.0 else 0.0)
+    out = []
+    for o in range(len(b2)):
+        acc = b2[o]
+        for u in range(len(hidden)):
+            acc += w2[o][u] * hidden[u]
+        out.append(acc)
+    return out
+
+
+def test_score_topk_assembly_by_explicit_loops():
+    """Which side is which in the score matrix, section 2.1: row i is Q tile i
+    (the Q-side MLP applied to the Q descriptor), column j is K tile j (the
+    K-side MLP applied to the K descriptor).  Q and K get different weights
+    and descriptors, the two heads have different tile counts, and B = 2, so
+    a transposed matrix, swapped weight sets, a swapped batch or head, or a
+    head read at the wrong NT all change the logits or the selection."""
+    grid, tilings, S = (3, 5, 7), [(1, 2, 4), (2, 2, 2)], 8
+    nts, ntmax = O.tile_layout(grid, tilings)
+    assert nts[0] != nts[1]
+    rng = np.random.default_rng(21)
+    B, heads, d3, hid, e = 2, 2, 9, 7, 5
+    dq = rng.standard_normal((B, heads, ntmax, d3))
+    dk = rng.standard_normal((B, heads, ntmax, d3)) * 1.3 + 0.2
+    mlp_q = (rng.standard_normal((heads, hid, d3)), rng.standard_normal((heads, hid)),
+             rng.standard_normal((heads, e, hid)), rng.standard_normal((heads, e)))
+    mlp_k = (rng.standard_normal((heads, hid, d3)), rng.standard_normal((heads, hid)),
+             rng.standard_normal((heads, e, hid)), rng.standard_normal((heads, e)))
+    keep = 0.3
+    idx, probs, scores = O.score_topk(dq, dk, grid, tilings, S, mlp_q, mlp_k, keep, want_scores=True)
+    for b in range(B):
+        for h in range(heads):
+            nt = nts[h]
+            k = O.keep_count(nt, keep)
+            wq = [m[h].tolist() for m in mlp_q]
+            wk = [m[h].tolist() for m in mlp_k]
+            phq = [_mlp_by_loops(dq[b, h, i].tolist(), *wq) for i in range(nt)]
+            phk = [_mlp_by_loops(dk[b, h, j].tolist(), *wk) for j in range(nt)]
+            for i in range(nt):
+                s = []
+                for j in range(nt):
+                    dot = 0.0
+                    for o in range(e):
+                        dot += phq[i][o] * phk[j][o]
+                    s.append(dot / math.sqrt(e))
+                np.testing.assert_allclose(scores[b, h, i, :nt], s, rtol=1e-11, atol=1e-11)
+                assert np.all(np.isneginf(scores[b, h, i, nt:]))
+                ref = sorted(sorted(range(nt), key=lambda j: (-s[j], j))[:k])
+                assert idx[b, h, i, :k].tolist() == ref, (b, h, i)
+                assert np.all(idx[b, h, i, k:] == -1)
+                z = [math.exp(v - max(s)) for v in s]
+                np.testing.assert_allclose(probs[b, h, i, :nt], [v / sum(z) for v in z], rtol=1e-12)
+            for i in range(nt, ntmax):
+                assert np.all(idx[b, h, i] == -1)
+
+
 # ---------------------------------------------------------------- step 5: attention
 def _inputs(grid, d, heads=2, seed=6):
     rng = np.random.default_rng(seed)
