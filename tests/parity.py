@@ -115,3 +115,18 @@ def mlp_device(m, device="cuda") -> tuple:
 def keep_f32(r: float) -> float:
     """The keep ratio as the C ABI receives it (a C float), widened back to double."""
     return float(np.float32(r))
+
+
+_QKV_CACHE = {}
+
+
+def cached_qkv(w: Workload, seed: int = 0):
+    """make_qkv(w, seed), kept for the test session: the full-size workloads
+    take tens of seconds to draw on the CPU and several test files use them.
+    Only the most recent workload is kept, to bound host memory."""
+    key = (w, seed)
+    if key not in _QKV_CACHE:
+        from veda_synth import make_qkv
+        _QKV_CACHE.clear()
+        _QKV_CACHE[key] = make_qkv(w, seed=seed)
+    return _QKV_CACHE[key]

@@ -78,3 +78,44 @@ def test_max_over_ranks_on_two_gloo_ranks():
     mp.spawn(_rank_main, args=(2, port, out), nprocs=2, join=True)
     assert dict(out) == {0: 15.0, 1: 15.0}
     assert bench.weak_scaling_value(7.8e12, 15.0, 2) == pytest.approx(2 * 7.8e12 / 15e-3 / 1e12)
+
+
+def _smi_line(ts, sm, mx=1965, pw=500.0, cap="Not Active"):
+    return (f"{ts}, 0, {sm}, {mx}, {pw}, 0x0000000000000000, Not Active, Not Active, Not Active, {cap}")
+
+
+def test_clock_summary_keeps_only_the_timed_region():
+    import datetime
+    base = datetime.datetime(2026, 12, 2, 12, 0, 0)
+    lines = []
+    for i in range(20):                       # one sample every 50 ms, 1 s in all
+        t = base + datetime.timedelta(milliseconds=50 * i)
+        sm = 1965 if 6 <= i <= 9 else 1400    # the region runs at full clock, the rest does not
+        lines.append(_smi_line(t.strftime("%Y/%m/%d %H:%M:%S.%f")[:-3], sm, cap="Active" if i > 15 else "Not Active"))
+    rows = bench.Clocks.parse(lines)
+    assert len(rows) == 20
+    t0 = (base + datetime.timedelta(milliseconds=290)).timestamp()
+    t1 = (base + datetime.timedelta(milliseconds=460)).timestamp()
+    clk = bench.Clocks.summarize(rows, t0, t1)
+    assert clk["samples"] == 4 and clk["sm_mhz"] == 1965 and clk["reasons"] == []
+    # a region shorter than the sampling interval takes the first sample after its start
+    t0 = (base + datetime.timedelta(milliseconds=810)).timestamp()
+    clk = bench.Clocks.summarize(rows, t0, t0 + 0.01)
+    assert clk["samples"] == 1 and clk["sm_mhz"] == 1400 and clk["reasons"] == ["sw_power_cap"]
+
+
+def test_peak_follows_the_clock_record():
+    peaks = {"bf16_tflops": 1674.3, "bf16_tflops_sustained": 1409.4, "hbm_gbs": 6541.8}
+    at_max = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 3, "window": "timed region"}
+    capped = {"sm_mhz": 1597.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 30,
+              "window": "timed region"}
+    assert bench.choose_peak(peaks, at_max, "measured")[0] == 1674.3
+    peak, basis = bench.choose_peak(peaks, capped, "measured")
+    assert peak == 1409.4 and "sustained" in basis and "sw_power_cap" in basis
+    assert bench.choose_peak(peaks, None, "measured")[0] == 1674.3
+
+
+def test_loglog_slope():
+    xs = [61440, 122880, 245760]
+    assert bench.loglog_slope(xs, [2.0 * x for x in xs]) == pytest.approx(1.0)
+    assert bench.loglog_slope(xs, [3e-9 * x * x for x in xs]) == pytest.approx(2.0)

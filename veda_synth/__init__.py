@@ -147,6 +147,30 @@ def make_qkv(w: Workload, seed: int = 0, heads: Optional[int] = None):
             torch.stack(vs, 1).contiguous())
 
 
+def make_qkv_on_device(w: Workload, device, seed: int = 0):
+    """The recipe of ``make_qkv`` drawn on ``device`` (bf16 [B, heads, N, d]
+    grid-order Q, K, V): N(0,1) values, plus the same kind of positional
+    feature on channels 0..15 of Q and K when ``w.bias`` is set.  The values
+    differ from ``make_qkv``'s (another generator); this is for timing runs at
+    sizes whose CPU draw would take longer than the measurement itself."""
+    dev = torch.device(device)
+    shape = (w.B, w.N, w.d)
+    feats = None
+    if w.bias is not None:
+        feats = _bias_features(w, torch.Generator().manual_seed(seed * 7919 + 17))
+    c = math.sqrt(4.0 * math.sqrt(w.d))
+    out = [torch.empty((w.B, w.heads, w.N, w.d), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    for h in range(w.heads):
+        g = torch.Generator(device=dev).manual_seed(seed * 100003 + h)
+        for a, t in enumerate(out):
+            x = torch.randn(shape, generator=g, device=dev)
+            if feats is not None and a < 2:
+                r = feats.shape[-1]
+                x[..., :r] += c * feats[h].to(dev)
+            t[:, h] = x.to(torch.bfloat16)
+    return tuple(out)
+
+
 def make_grad_out(w: Workload, seed: int = 4, heads: Optional[int] = None) -> torch.Tensor:
     """An upstream gradient dO for the attention backward: bf16 CPU tensor
     [B, heads, N, d] in grid order, N(0,1) drawn in fp32 per head from its own
