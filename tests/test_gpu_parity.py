@@ -14,8 +14,8 @@ import torch
 from oracle import veda_oracle as O
 from veda_synth import PRESETS, make_map_rows, make_mlp, make_qkv
 
-from parity import (LSE_ABS, MAP_REL, MEAN_REL, PROBS_ABS, PROBS_REL, SMALL, check_attn_rows, check_idx, f64,
-                    keep_f32, mlp_device, mlp_numpy)
+from parity import (LSE_ABS, MAP_REL, MEAN_REL, PROBS_ABS, PROBS_REL, SMALL, cached_qkv, check_attn_rows, check_idx,
+                    f64, keep_f32, mlp_device, mlp_numpy)
 
 pytestmark = pytest.mark.gpu
 
@@ -206,7 +206,7 @@ def test_wan14b_full_size_sampled(V):
     """Wan2.1-14B 720p/81-frame shape at keep 5%, the benchmarked launch, on sampled heads and tiles."""
     w = PRESETS["wan14b"]
     p = _problem(V, w)
-    q, k, v = make_qkv(w, seed=0)
+    q, k, v = cached_qkv(w, 0)
     m = make_mlp(w, seed=1)
     att = V.VedaAttention(p, mlp_device(m), mlp_device(m), w.keep, want_lse=True, layout="tile")
     out = att(q.cuda(), k.cuda(), v.cuda())
