@@ -59,7 +59,8 @@ typedef enum {
   VEDA_ERR_INVALID_ARG = 1,   /* bad pointer, size, ratio or tiling */
   VEDA_ERR_UNSUPPORTED = 2,   /* valid request outside the built shapes (d, S) */
   VEDA_ERR_CUDA = 3,          /* a CUDA runtime call or a launch failed */
-  VEDA_ERR_TIMEOUT = 4        /* a kernel gave up on a bounded wait (device error word set) */
+  VEDA_ERR_TIMEOUT = 4,       /* a kernel gave up on a bounded wait (device error word set) */
+  VEDA_ERR_BOUNDS = 5         /* debug builds only: a kernel's index check failed and the access was skipped */
 } veda_status;
 
 /* Video token grid: frames T, height H, width W (latent tokens). */
@@ -186,7 +187,9 @@ veda_status veda_tile_score_topk(const veda_problem* p, const float* desc_q, con
  * veda_tile_score_topk).  This call allocates nothing.  Every GPU that loads
  * the library holds the array until the process exits.  The first call on a
  * device looks up the array's device address (cudaGetSymbolAddress) for that
- * device; make that first call before any stream capture.  All calls share
+ * device; make that first call before any stream capture.  The address is
+ * kept per device and per context: after cudaDeviceReset the next call looks
+ * it up again (so, again, not inside a capture).  All calls share
  * the one array, so calls that may overlap on the GPU (different streams,
  * or different host threads on one device) race: serialise them.  Nothing
  * needs clearing between calls -- every value read is written earlier in the
@@ -330,7 +333,10 @@ veda_status veda_tile_sparse_attn_backward_grid(const veda_problem* p, const voi
 
 /* Synchronises `stream`, then reads and clears the library's device error
  * word (set by a kernel that gave up on a bounded wait).  Returns VEDA_OK,
- * VEDA_ERR_TIMEOUT or VEDA_ERR_CUDA. */
+ * VEDA_ERR_TIMEOUT or VEDA_ERR_CUDA.  The error word is one per device and
+ * process, shared by every stream and thread: a status read through stream A
+ * can report (and clears) a fault raised by a kernel on stream B.  Callers
+ * that need per-stream attribution synchronise the other streams first. */
 veda_status veda_sync_status(void* stream);
 
 /* Limit of every bounded wait inside the library's kernels, in nanoseconds
@@ -344,6 +350,20 @@ veda_status veda_set_wait_timeout_ns(uint64_t ns);
  * `timeout_ns` ([1 us, 10 s]).  The following veda_sync_status(stream)
  * must report VEDA_ERR_TIMEOUT; the context stays usable. */
 veda_status veda_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
+
+/* 1 for a debug build (compiled with -DVEDA_DEBUG_BOUNDS: every index a
+ * kernel computes -- tile ids, tensor rows, selection entries -- is checked
+ * before use; a failed check skips the access, sets the device error word and
+ * veda_sync_status returns VEDA_ERR_BOUNDS naming the source line), 0 for a
+ * release build, where the checks compile away. */
+int32_t veda_bounds_checked(void);
+
+/* Bounds-check self-test (no counterpart on the pages; debug builds only):
+ * launches one tiny kernel whose last thread fails a bounds check and touches
+ * no memory.  The following veda_sync_status(stream) must return
+ * VEDA_ERR_BOUNDS.  A release build returns VEDA_ERR_UNSUPPORTED and launches
+ * nothing. */
+veda_status veda_selftest_bounds(void* stream);
 
 /* Thread-local text of the last failure ("" if none).  Valid until the next
  * call on this thread. */

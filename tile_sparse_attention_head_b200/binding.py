@@ -16,12 +16,14 @@ from typing import Optional, Sequence, Tuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libveda.so")
+# VEDA_DEBUG_BOUNDS=1 loads the debug build (build.py --debug), whose kernels
+# check every computed index and report a failed check as VEDA_ERR_BOUNDS.
+LIB_PATH = os.path.join(_HERE, "libveda_debug.so" if os.environ.get("VEDA_DEBUG_BOUNDS") == "1" else "libveda.so")
 
-VEDA_OK, VEDA_ERR_INVALID_ARG, VEDA_ERR_UNSUPPORTED, VEDA_ERR_CUDA, VEDA_ERR_TIMEOUT = range(5)
+VEDA_OK, VEDA_ERR_INVALID_ARG, VEDA_ERR_UNSUPPORTED, VEDA_ERR_CUDA, VEDA_ERR_TIMEOUT, VEDA_ERR_BOUNDS = range(6)
 MAX_HEADS = 128
 _STATUS_NAMES = {0: "VEDA_OK", 1: "VEDA_ERR_INVALID_ARG", 2: "VEDA_ERR_UNSUPPORTED", 3: "VEDA_ERR_CUDA",
-                 4: "VEDA_ERR_TIMEOUT"}
+                 4: "VEDA_ERR_TIMEOUT", 5: "VEDA_ERR_BOUNDS"}
 
 
 class VedaError(RuntimeError):
@@ -84,12 +86,16 @@ _SIG = {
     "veda_sync_status": [_V],
     "veda_set_wait_timeout_ns": [ctypes.c_uint64],
     "veda_selftest_wait_timeout": [ctypes.c_uint64, _V],
+    "veda_selftest_bounds": [_V],
+    "veda_bounds_checked": [],
 }
 
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libveda.so is not built ({LIB_PATH}); run tile_sparse_attention_head_b200/build.py")
+        raise ImportError(f"{os.path.basename(LIB_PATH)} is not built ({LIB_PATH}); "
+                          "run tile_sparse_attention_head_b200/build.py" +
+                          (" --debug" if LIB_PATH.endswith("_debug.so") else ""))
     lib = ctypes.CDLL(LIB_PATH)
     for name, args in _SIG.items():
         fn = getattr(lib, name)
@@ -385,6 +391,17 @@ def veda_set_wait_timeout_ns(ns: int) -> None:
 
 def veda_selftest_wait_timeout(timeout_ns: int, stream=None) -> None:
     _check(LIB.veda_selftest_wait_timeout(int(timeout_ns), _stream(stream)), "veda_selftest_wait_timeout")
+
+
+def veda_bounds_checked() -> bool:
+    """True when the loaded library is the debug build with device-side index checks."""
+    return bool(LIB.veda_bounds_checked())
+
+
+def veda_selftest_bounds(stream=None) -> None:
+    """Debug builds: one kernel fails a bounds check on purpose (no memory is
+    touched); the next veda_sync_status raises VEDA_ERR_BOUNDS."""
+    _check(LIB.veda_selftest_bounds(_stream(stream)), "veda_selftest_bounds")
 
 
 def veda_version() -> str:

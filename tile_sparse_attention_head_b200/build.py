@@ -14,6 +14,10 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libveda.so")
+# Debug build: every computed index is checked in the kernels (-DVEDA_DEBUG_BOUNDS);
+# a failed check is reported by veda_sync_status as VEDA_ERR_BOUNDS.  The
+# binding loads it instead of LIB when VEDA_DEBUG_BOUNDS=1 is set.
+DEBUG_LIB = os.path.join(HERE, "libveda_debug.so")
 SOURCES = ["veda_api.cu", "veda_common.cuh", "kernels.h", "permute_tripool.cu", "score_topk.cu",
            "sparse_attn.cu", "tile_map.cu", "estimator.cu", "distill.cu", "attn_bwd.cu"]
 
@@ -31,28 +35,38 @@ def nvcc_command(out: str = LIB, extra=()) -> list:
             "-o", out, os.path.join(CSRC, "veda_api.cu")]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, s) for s in SOURCES] + [os.path.join(HERE, "..", "include", "veda.h")]
     return all(os.path.getmtime(p) <= t for p in deps if os.path.exists(p))
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = nvcc_command(tmp, ["-Xptxas", "-v"] if verbose else [])
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib = DEBUG_LIB if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    tmp = lib + ".tmp"
+    extra = (["-Xptxas", "-v"] if verbose else []) + (["-DVEDA_DEBUG_BOUNDS"] if debug else [])
+    cmd = nvcc_command(tmp, extra)
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError("nvcc failed building libveda.so")
+        raise RuntimeError(f"nvcc failed building {os.path.basename(lib)}")
     if verbose:
         sys.stderr.write(res.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build_all(force: bool = False) -> list:
+    """The release library and the debug (bounds-checked) one, compiled side by side."""
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(2) as ex:
+        futs = [ex.submit(build, force, False, dbg) for dbg in (False, True)]
+        return [f.result() for f in futs]
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug="--debug" in sys.argv))

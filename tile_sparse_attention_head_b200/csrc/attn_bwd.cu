@@ -48,6 +48,8 @@
 // copies and products are drained and TMEM is freed.
 #include "veda_common.cuh"
 #include "kernels.h"
+#undef VEDA_SRC_ID
+#define VEDA_SRC_ID 6   // bounds-check site id of this file (debug builds)
 
 namespace veda {
 
@@ -192,6 +194,7 @@ __global__ void __launch_bounds__(384, 1)
   for (int c = tid; c < n_list; c += C::kThreads) {
     const int v = mov[c];
     if (!KV && (v < 0 || v >= hg.nt)) atomicMin(&misc[2], c);
+    if (KV) (void)VEDA_IN_BOUNDS(v >= 0 && v < hg.nt);   // the inverse lists hold Q tiles of this head
     if (c < C::kListCap) s_list[c] = (int16_t)v;
   }
   if (tid == 0) {
@@ -508,7 +511,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) a[e] = 0.f;
         }
-        if (rvalid) {
+        if (rvalid && VEDA_IN_BOUNDS(n_row >= 0 && n_row < G.N)) {
           uint4* dst = reinterpret_cast<uint4*>(out + ((long long)bh * G.N + n_row) * D + d0 + 32 * q);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4) {

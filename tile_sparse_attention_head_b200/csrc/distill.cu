@@ -28,6 +28,8 @@
 #pragma once
 #include "veda_common.cuh"
 #include "kernels.h"
+#undef VEDA_SRC_ID
+#define VEDA_SRC_ID 7   // bounds-check site id of this file (debug builds)
 
 namespace veda {
 

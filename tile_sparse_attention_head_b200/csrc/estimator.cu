@@ -29,6 +29,8 @@
 #pragma once
 #include "veda_common.cuh"
 #include "kernels.h"
+#undef VEDA_SRC_ID
+#define VEDA_SRC_ID 3   // bounds-check site id of this file (debug builds)
 
 namespace veda {
 
@@ -245,7 +247,7 @@ __global__ void __launch_bounds__(kEstThreads, 1)
       float v[32];
       tmem_ld32(tmem + kEstAcc2 + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
       tmem_ld_wait();
-      if (r < nrows) {
+      if (r < nrows && VEDA_IN_BOUNDS(j0 + r < G.ntmax)) {
 #pragma unroll
         for (int q = 0; q < 32 && c0 + q < E; q += 4) {
           float4 o4 = make_float4(v[q] + __ldg(B2 + c0 + q), v[q + 1] + __ldg(B2 + c0 + q + 1),

@@ -130,5 +130,6 @@ cudaError_t launch_attn_bwd_dkdv(const Geometry& G, const BwdMaps<kMaxGridMaps>&
                                  cudaStream_t s);
 
 cudaError_t launch_timeout_selftest(uint64_t timeout_ns, cudaStream_t s);
+cudaError_t launch_bounds_selftest(cudaStream_t s);
 
 }  // namespace veda

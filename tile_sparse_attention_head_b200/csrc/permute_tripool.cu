@@ -19,6 +19,8 @@
 // with several loads in flight per thread.
 #include "veda_common.cuh"
 #include "kernels.h"
+#undef VEDA_SRC_ID
+#define VEDA_SRC_ID 1   // bounds-check site id of this file (debug builds)
 
 namespace veda {
 
@@ -137,12 +139,14 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(const __grid_
       v[u] = make_uint4(0u, 0u, 0u, 0u);
       if (ok[u]) {
         const size_t row = SRC_GRID ? ((size_t)(t0 + ot) * G.H + (y0 + oh)) * G.W + (x0 + ow) : (size_t)l;
-        v[u] = __ldg(sb + row * CPR);
+        if (VEDA_IN_BOUNDS(row < (SRC_GRID ? (size_t)G.N : (size_t)S))) v[u] = __ldg(sb + row * CPR);
       }
     }
 #pragma unroll
     for (int u = 0; u < UNR; ++u) {
-      if constexpr (WRITE) xo[(size_t)((s0 + u) * RPI + r0) * CPR] = v[u];
+      if constexpr (WRITE) {
+        if (VEDA_IN_BOUNDS((s0 + u) * RPI + r0 < S)) xo[(size_t)((s0 + u) * RPI + r0) * CPR] = v[u];
+      }
       if constexpr (POOL) {
         if (ok[u]) st8.add(v[u]);
       }
@@ -178,11 +182,12 @@ __global__ void __launch_bounds__(kPermThreads) unpermute_kernel(const __grid_co
 #pragma unroll
   for (int p = 0; p < PASSES; ++p) {
     const int pos = s_pos[r0 + p * RPP];
-    if (pos >= 0) v[p] = __ldg(xi + (size_t)pos * CPR + chunk);
+    if (pos >= 0 && VEDA_IN_BOUNDS(pos < G.ntmax * G.S)) v[p] = __ldg(xi + (size_t)pos * CPR + chunk);
   }
 #pragma unroll
   for (int p = 0; p < PASSES; ++p)
-    if (s_pos[r0 + p * RPP] >= 0) xo[(size_t)(r0 + p * RPP) * CPR + chunk] = v[p];
+    if (s_pos[r0 + p * RPP] >= 0 && VEDA_IN_BOUNDS(n0 + r0 + p * RPP < G.N))
+      xo[(size_t)(r0 + p * RPP) * CPR + chunk] = v[p];
 }
 
 template <bool SRC_GRID, bool WRITE, bool POOL>

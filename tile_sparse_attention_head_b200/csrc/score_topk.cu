@@ -21,6 +21,8 @@
 #include "veda_common.cuh"
 #include "kernels.h"
 #include "estimator.cu"
+#undef VEDA_SRC_ID
+#define VEDA_SRC_ID 2   // bounds-check site id of this file (debug builds)
 
 namespace veda {
 
@@ -163,7 +165,8 @@ __global__ void __launch_bounds__(kScoreThreads)
       if (r < nrows) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-          if (4 * cg + c < ncols) s_scores[r * ntpad + jc + 4 * cg + c] = acc[q][c] * inv_sqrt_e;
+          if (4 * cg + c < ncols && VEDA_IN_BOUNDS(jc + 4 * cg + c < ntpad))
+            s_scores[r * ntpad + jc + 4 * cg + c] = acc[q][c] * inv_sqrt_e;
       }
     }
   }
@@ -276,7 +279,7 @@ __global__ void __launch_bounds__(kScoreThreads)
       const bool take = gt || (eq && eq_taken + eq_before < remaining);
       const unsigned tmask = __ballot_sync(0xffffffffu, take);
       const int pos = out + __popc(tmask & ((1u << lane) - 1u));
-      if (take && pos < k) irow[pos] = c;
+      if (take && pos < k && VEDA_IN_BOUNDS(c < nt && pos < args.k_max)) irow[pos] = c;
       out += __popc(tmask);
       eq_taken += __popc(eqmask);
     }

@@ -37,6 +37,8 @@
 // its loop, in-flight copies and MMAs are drained and TMEM is freed.
 #include "veda_common.cuh"
 #include "kernels.h"
+#undef VEDA_SRC_ID
+#define VEDA_SRC_ID 4   // bounds-check site id of this file (debug builds)
 
 namespace veda {
 
@@ -270,9 +272,11 @@ __global__ void __launch_bounds__(384, 1)
         if (fill >= 1 && !warp_wait(bar(BAR_KEMPTY + st), (fill - 1) & 1, abort, tmo)) break;
         if (lane == 0) {
           const int j = s_idx[t];
-          mbar_arrive_expect_tx(bar(BAR_KFULL + st), (uint32_t)C::kTileBytes);
-          for (int c = 0; c < D / 64; ++c)
-            load_tile(sK + st * C::kTileBytes + c * BN * 128, tmK, bar(BAR_KFULL + st), c, j);
+          if (VEDA_IN_BOUNDS(j >= 0 && j < hg.nt)) {   // a skipped fetch runs the consumers' waits out
+            mbar_arrive_expect_tx(bar(BAR_KFULL + st), (uint32_t)C::kTileBytes);
+            for (int c = 0; c < D / 64; ++c)
+              load_tile(sK + st * C::kTileBytes + c * BN * 128, tmK, bar(BAR_KFULL + st), c, j);
+          }
         }
         __syncwarp();
         issued = t + 1;
@@ -293,9 +297,11 @@ __global__ void __launch_bounds__(384, 1)
         if (fill >= 1 && !warp_wait(bar(BAR_VEMPTY + st), (fill - 1) & 1, abort, tmo)) break;
         if (lane == 0) {
           const int j = s_idx[t];
-          mbar_arrive_expect_tx(bar(BAR_VFULL + st), (uint32_t)C::kTileBytes);
-          for (int c = 0; c < D / 64; ++c)
-            load_tile(sV + st * C::kTileBytes + c * BN * 128, tmV, bar(BAR_VFULL + st), c, j);
+          if (VEDA_IN_BOUNDS(j >= 0 && j < hg.nt)) {
+            mbar_arrive_expect_tx(bar(BAR_VFULL + st), (uint32_t)C::kTileBytes);
+            for (int c = 0; c < D / 64; ++c)
+              load_tile(sV + st * C::kTileBytes + c * BN * 128, tmV, bar(BAR_VFULL + st), c, j);
+          }
         }
         __syncwarp();
         issued = t + 1;
@@ -524,6 +530,7 @@ __global__ void __launch_bounds__(384, 1)
       } else {
         grow = ((long long)bh * G.ntmax + i) * S + row;
       }
+      if (valid) valid = VEDA_IN_BOUNDS(grow < (long long)G.B * G.heads * (GRID ? (long long)G.N : (long long)G.ntmax * S));
       uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(A.op) + grow * D + s * (D / 2));
 #pragma unroll
       for (int c = 0; c < D / 2; c += 32) {

@@ -24,6 +24,8 @@
 // than re-running the tensor-core sweep.
 #include "veda_common.cuh"
 #include "kernels.h"
+#undef VEDA_SRC_ID
+#define VEDA_SRC_ID 5   // bounds-check site id of this file (debug builds)
 
 namespace veda {
 
@@ -135,7 +137,7 @@ __global__ void __launch_bounds__(320, 1)
       const int st = t % C::kStages;
       const int fill = t / C::kStages;
       if (fill >= 1 && !map_warp_wait(bar(MBAR_KEMPTY + st), (fill - 1) & 1, abort, tmo)) break;
-      if (lane == 0) {
+      if (lane == 0 && VEDA_IN_BOUNDS(t < hg.nt && (long long)(bh * G.ntmax + t) * S < (long long)G.B * G.heads * G.ntmax * S)) {
         mbar_arrive_expect_tx(bar(MBAR_KFULL + st), (uint32_t)C::kKBytes);
         for (int c = 0; c < D / 64; ++c)
           tma_load_2d(sK + st * C::kKBytes + c * BN * 128, &tmK, bar(MBAR_KFULL + st), 64 * c,
@@ -245,7 +247,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int q = 0; q < 8; ++q) m8[q] = fmaxf(m8[q], sc[BN - 8 + q]);
       }
       const float mt = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * sl2;
-      if (row < S) rm[(long long)t * S] = mt;
+      if (row < S && VEDA_IN_BOUNDS(t < nt)) rm[(long long)t * S] = mt;
       const float m_new = fmaxf(m_run, mt);
       const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
       const uint64_t nref2 = f2(-m_ref, -m_ref);
@@ -321,7 +323,7 @@ __global__ void __launch_bounds__(256) tile_map_pass2_kernel(const __grid_consta
       for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
       best = exp2f(m);
     }
-    if (lane == 0) A.map[w] = best;
+    if (lane == 0 && VEDA_IN_BOUNDS(w < total)) A.map[w] = best;
   }
 }
 
@@ -371,6 +373,15 @@ __global__ void timeout_selftest_kernel(uint64_t timeout_ns) {
 
 cudaError_t launch_timeout_selftest(uint64_t timeout_ns, cudaStream_t s) {
   timeout_selftest_kernel<<<1, 32, 0, s>>>(timeout_ns);
+  return cudaGetLastError();
+}
+
+// Bounds-check self-test (debug builds): thread t checks t < limit, the way
+// the kernels check a computed index, and touches no memory.
+__global__ void bounds_selftest_kernel(int limit) { (void)VEDA_IN_BOUNDS((int)threadIdx.x < limit); }
+
+cudaError_t launch_bounds_selftest(cudaStream_t s) {
+  bounds_selftest_kernel<<<1, 32, 0, s>>>(31);
   return cudaGetLastError();
 }
 

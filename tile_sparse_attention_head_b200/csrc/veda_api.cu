@@ -353,22 +353,56 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
 
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device (the host-side symbol is only a stand-in, never a device pointer).
+// Unique id of the calling thread's current CUDA context, or 0 when none is
+// current (or the driver predates cuCtxGetId).  Ids are never reused within a
+// process, so a context torn down by cudaDeviceReset and created again gets a
+// new one.
+unsigned long long current_context_id() {
+  using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+  using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_noalloc_scratch on the current device.  It is looked
+// up once per device and context (the host-side symbol is only a stand-in,
+// never a device pointer) and looked up again when the device's context has
+// changed since, e.g. after cudaDeviceReset.
 veda_status noalloc_scratch(float** out) {
   constexpr int kMaxDevices = 64;
   static float* ptrs[kMaxDevices] = {};
+  static unsigned long long ctx_ids[kMaxDevices] = {};
   static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "veda_tile_score_topk_noalloc: cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(VEDA_ERR_UNSUPPORTED, "device ordinal %d above %d", dev, kMaxDevices - 1);
   std::lock_guard<std::mutex> lock(mu);
-  if (ptrs[dev] == nullptr) {
+  const unsigned long long id = current_context_id();
+  if (ptrs[dev] == nullptr || id == 0 || id != ctx_ids[dev]) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);   // also makes the device's primary context current
     if (e != cudaSuccess) return cuda_fail(e, "veda_tile_score_topk_noalloc: cudaGetSymbolAddress");
     ptrs[dev] = static_cast<float*>(p);
+    ctx_ids[dev] = current_context_id();
   }
   *out = ptrs[dev];
   return VEDA_OK;
@@ -733,10 +767,20 @@ veda_status veda_sync_status(void* stream) {
   e = cudaMemcpyFromSymbol(&word, g_device_error, sizeof(int));
   if (e != cudaSuccess) return cuda_fail(e, "veda_sync_status: read device error word");
   if (word != kErrNone) {
+    int site = 0;
+    if (word == kErrBounds) cudaMemcpyFromSymbol(&site, g_bounds_site, sizeof(int));
     const int zero = 0;
     cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+    cudaMemcpyToSymbol(g_bounds_site, &zero, sizeof(int));
     if (word == kErrSmemAlign)
       return fail(VEDA_ERR_CUDA, "a kernel found its dynamic shared memory base not 1024-byte aligned");
+    if (word == kErrBounds) {
+      static const char* const files[] = {"?", "permute_tripool.cu", "score_topk.cu", "estimator.cu",
+                                          "sparse_attn.cu", "tile_map.cu", "attn_bwd.cu", "distill.cu"};
+      const int f = site / 10000;
+      return fail(VEDA_ERR_BOUNDS, "debug bounds check failed at %s:%d; the access was skipped",
+                  files[(f >= 0 && f < 8) ? f : 0], site % 10000);
+    }
     return fail(VEDA_ERR_TIMEOUT, "a kernel gave up on a bounded wait (device error word %d)", word);
   }
   return ok();
@@ -754,6 +798,25 @@ veda_status veda_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
   cudaError_t e = launch_timeout_selftest(timeout_ns, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "veda_selftest_wait_timeout");
   return ok();
+}
+
+int32_t veda_bounds_checked(void) {
+#ifdef VEDA_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+veda_status veda_selftest_bounds(void* stream) {
+#ifdef VEDA_DEBUG_BOUNDS
+  cudaError_t e = launch_bounds_selftest((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "veda_selftest_bounds");
+  return ok();
+#else
+  (void)stream;
+  return fail(VEDA_ERR_UNSUPPORTED, "veda_selftest_bounds: this library is a release build without bounds checks");
+#endif
 }
 
 }  // extern "C"

@@ -70,8 +70,27 @@ __device__ __forceinline__ int tile_token_count(const Geometry& G, const HeadGeo
 // Device error word: kernels that give up on a bounded wait record a code here
 // and return; veda_sync_status() reads and clears it.
 // ----------------------------------------------------------------------------
-enum : int { kErrNone = 0, kErrTimeout = 1, kErrSmemAlign = 2 };
+enum : int { kErrNone = 0, kErrTimeout = 1, kErrSmemAlign = 2, kErrBounds = 3 };
 __device__ int g_device_error = 0;
+// Site of the first failed bounds check (debug builds): source id * 10000 +
+// line, the source ids being the VEDA_SRC_ID values of the kernel files.
+__device__ int g_bounds_site = 0;
+
+// Debug builds (compiled with -DVEDA_DEBUG_BOUNDS, build.py --debug) check
+// every index a kernel computes before it uses it: a tile id against the
+// head's tile count, a row against the tensor's rows, a selection entry
+// against [0, NT_h).  A failed check records its site and the error word and
+// the access is skipped; nothing traps, and veda_sync_status reports
+// VEDA_ERR_BOUNDS.  Release builds compile the checks away.
+#ifdef VEDA_DEBUG_BOUNDS
+__device__ __forceinline__ bool bounds_ok(bool c, int site) {
+  if (!c && atomicCAS(&g_device_error, kErrNone, kErrBounds) == kErrNone) atomicExch(&g_bounds_site, site);
+  return c;
+}
+#define VEDA_IN_BOUNDS(cond) (::veda::bounds_ok((cond), VEDA_SRC_ID * 10000 + __LINE__))
+#else
+#define VEDA_IN_BOUNDS(cond) (true)
+#endif
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -129,7 +148,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (*abort) return false;
     if (globaltimer_ns() - t0 > timeout_ns) {
       *abort = 1;
-      atomicExch(&g_device_error, kErrTimeout);
+      atomicCAS(&g_device_error, kErrNone, kErrTimeout);   // the first error recorded is kept
       return false;
     }
   }
