@@ -177,18 +177,16 @@ class Clocks:
 
 def choose_peak(peaks, clk, peak_src):
     """The tensor peak a kernel timed in this run is held against.  The burst
-    figure (a GEMM timed alone, at full clock) applies when the SM clock in the
-    timed region sat at its maximum; the sustained figure (a GEMM run for
-    seconds at the board's power cap) applies when the power cap held the
-    clock down.  Returns (peak, basis)."""
+    figure (a GEMM timed alone, at full clock) applies unless the clock record
+    of the timed region shows the board's power cap (or a thermal or hardware
+    slowdown) holding the clock down; then the sustained figure (a GEMM run for
+    seconds at the power cap) applies.  Returns (peak, basis)."""
     if clk is not None and clk.get("sm_mhz") and clk.get("sm_max_mhz"):
-        at_max = clk["sm_mhz"] >= 0.97 * clk["sm_max_mhz"]
         basis = (f"median SM clock {clk['sm_mhz']:.0f} of {clk['sm_max_mhz']:.0f} MHz over "
-                 f"{clk['samples']} sample(s) in the {clk.get('window', 'run')}")
-        if at_max:
+                 f"{clk['samples']} sample(s) in the {clk.get('window', 'run')}, reasons {clk['reasons']}")
+        if not clk["reasons"]:
             return peaks["bf16_tflops"], f"{peak_src} bf16 burst: {basis}"
-        return peaks["bf16_tflops_sustained"], (f"{peak_src} bf16 sustained (power-capped GEMM): {basis}, "
-                                                f"reasons {clk['reasons']}")
+        return peaks["bf16_tflops_sustained"], f"{peak_src} bf16 sustained (power-capped GEMM): {basis}"
     return peaks["bf16_tflops"], f"{peak_src} bf16 burst (no clock record)"
 
 

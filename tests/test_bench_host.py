@@ -113,6 +113,9 @@ def test_peak_follows_the_clock_record():
     peak, basis = bench.choose_peak(peaks, capped, "measured")
     assert peak == 1409.4 and "sustained" in basis and "sw_power_cap" in basis
     assert bench.choose_peak(peaks, None, "measured")[0] == 1674.3
+    # below the maximum with no reason recorded: the burst figure still applies
+    low = dict(at_max, sm_mhz=1852.0)
+    assert bench.choose_peak(peaks, low, "measured")[0] == 1674.3
 
 
 def test_loglog_slope():
