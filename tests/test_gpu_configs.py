@@ -117,17 +117,17 @@ def test_topk_sweep246k_sampled_heads(V):
 
 
 # ------------------------------------------------------------------ attention ring depths
-RING32 = wl("dense128", (7, 30, 60), 1, 1, 128, 128, [(2, 8, 8)], 1.0, 256, 64, "rff")
+RING32 = wl("dense192", (11, 30, 64), 1, 1, 128, 128, [(2, 8, 8)], 1.0, 256, 64, "rff")
 
 
 @pytest.mark.parametrize("layout", ["tile", "grid"])
 def test_attention_three_k_two_v_stages_full_keep(V, layout):
-    """128 tiles, all kept: the selection list is long enough that the launch
+    """192 tiles, all kept: the selection list is long enough that the launch
     takes 3 K stages and 2 V stages; the whole output against the oracle."""
     w = RING32
     p = _problem(V, w)
     ks, k_max = p.keep_count(w.keep)
-    assert k_max == p.nt_max == 128
+    assert k_max == p.nt_max == 192
     kst, vst, _ = V.veda_attn_config(p, k_max)
     assert (kst, vst) == (3, 2)
     q, k, v = make_qkv(w, seed=2)
@@ -137,7 +137,7 @@ def test_attention_three_k_two_v_stages_full_keep(V, layout):
     out = att(q.cuda(), k.cuda(), v.cuda())
     V.veda_sync_status()
     gi = att.idx.cpu().numpy()
-    assert np.array_equal(gi[0, 0], np.tile(np.arange(128, dtype=np.int32), (128, 1)))
+    assert np.array_equal(gi[0, 0], np.tile(np.arange(192, dtype=np.int32), (192, 1)))
     grid = (w.T, w.H, w.W)
     qd, kd, vd = (f64(t) for t in (q, k, v))
     perm = [O.tile_permute(a, grid, w.tilings, w.S) for a in (qd, kd, vd)]
