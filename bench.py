@@ -56,7 +56,7 @@ WORKLOAD_NAMES = {"wan14b": "Wan2.1-14B-720p-81f 21x45x80 (75,600 tokens) 40 hea
 # keyed by workload and layout and tied to the kernel source it was measured
 # on: reported only while csrc/sparse_attn.cu still hashes to that version.
 ATTN_TRAFFIC = {("wan14b", "tile"): {"bytes": 1.26e9 + 858.49e6, "src_sha256_16": "b5a8f826b6c7f91f"},
-                ("wan14b", "grid"): {"bytes": 1.16e9 + 740.13e6, "src_sha256_16": "162ba4dc4a828fde"}}
+                ("wan14b", "grid"): {"bytes": 1139.32e6 + 740.37e6, "src_sha256_16": "1805a41c0b164c3f"}}
 
 
 def attn_traffic(workload: str, layout: str):
