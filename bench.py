@@ -179,12 +179,14 @@ def choose_peak(peaks, clk, peak_src):
     """The tensor peak a kernel timed in this run is held against.  The burst
     figure (a GEMM timed alone, at full clock) applies unless the clock record
     of the timed region shows the board's power cap (or a thermal or hardware
-    slowdown) holding the clock down; then the sustained figure (a GEMM run for
-    seconds at the power cap) applies.  Returns (peak, basis)."""
+    slowdown) holding the clock down -- a throttle reason present and the
+    median SM clock below its maximum; then the sustained figure (a GEMM run
+    for seconds at the power cap) applies.  Returns (peak, basis)."""
     if clk is not None and clk.get("sm_mhz") and clk.get("sm_max_mhz"):
         basis = (f"median SM clock {clk['sm_mhz']:.0f} of {clk['sm_max_mhz']:.0f} MHz over "
                  f"{clk['samples']} sample(s) in the {clk.get('window', 'run')}, reasons {clk['reasons']}")
-        if not clk["reasons"]:
+        held_down = bool(clk["reasons"]) and clk["sm_mhz"] < 0.97 * clk["sm_max_mhz"]
+        if not held_down:
             return peaks["bf16_tflops"], f"{peak_src} bf16 burst: {basis}"
         return peaks["bf16_tflops_sustained"], f"{peak_src} bf16 sustained (power-capped GEMM): {basis}"
     return peaks["bf16_tflops"], f"{peak_src} bf16 burst (no clock record)"
@@ -265,15 +267,21 @@ def useful_flops(w, idx):
 
 
 def tile_map_measure(V, w, p, qd, kd, args, rank, att=None):
-    """Times veda_tile_map_maxpool over a random 10% of Q tiles per head (the
-    distillation target), with its tensor and exponential bounds."""
+    """Times the max-pooled tile map over a random 10% of Q tiles per head (the
+    distillation target), with its tensor and exponential bounds: on the
+    grid-order tensors (veda_tile_map_maxpool_grid) with --layout grid, on
+    permuted copies (veda_tile_map_maxpool) with --layout tile."""
     from veda_synth import make_map_rows
     dev = qd.device
-    ts = p.tile_shape()
-    qp = torch.empty(ts, dtype=torch.bfloat16, device=dev)
-    kp = torch.empty(ts, dtype=torch.bfloat16, device=dev)
-    V.veda_tile_permute(p, qd, qp)
-    V.veda_tile_permute(p, kd, kp)
+    if args.layout == "grid":
+        qm, km, map_call = qd, kd, V.veda_tile_map_maxpool_grid
+    else:
+        ts = p.tile_shape()
+        qm = torch.empty(ts, dtype=torch.bfloat16, device=dev)
+        km = torch.empty(ts, dtype=torch.bfloat16, device=dev)
+        V.veda_tile_permute(p, qd, qm)
+        V.veda_tile_permute(p, kd, km)
+        map_call = V.veda_tile_map_maxpool
     rows = make_map_rows(p.nt_per_head, w.B, 0.1, seed=2)
     R = rows.shape[1]
     counts = (rows >= 0).sum(dim=1).view(w.B, w.heads).numpy()
@@ -281,13 +289,13 @@ def tile_map_measure(V, w, p, qd, kd, args, rank, att=None):
     ws = torch.empty(V.veda_tile_map_workspace(p, R) // 4 + 64, dtype=torch.float32, device=dev)
     mp = torch.empty((w.B, w.heads, R, p.nt_max), dtype=torch.float32, device=dev)
     for _ in range(2):
-        V.veda_tile_map_maxpool(p, qp, kp, rows, mp, ws)
+        map_call(p, qm, km, rows, mp, ws)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.map_steps):
-        V.veda_tile_map_maxpool(p, qp, kp, rows, mp, ws)
+        map_call(p, qm, km, rows, mp, ws)
     e1.record()
     torch.cuda.synchronize()
     V.veda_sync_status()
@@ -321,7 +329,7 @@ def tile_map_measure(V, w, p, qd, kd, args, rank, att=None):
     peaks, src = load_peaks()
     tflops = flops / (ms * 1e-3) / 1e12
     mufu_peak = 16 * 148 * peaks.get("sm_max_mhz", 1965.0) * 1e6   # ex2 per second at the maximum clock
-    return {"ms": ms, "subset_rows": int(counts.sum()), "flops": flops, "exps": exps, "tflops": tflops,
+    return {"ms": ms, "layout": args.layout, "subset_rows": int(counts.sum()), "flops": flops, "exps": exps, "tflops": tflops,
             "distill_step": dist,
             "roofline": {"bound": "tensor+exp", "achieved": tflops, "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],

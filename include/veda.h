@@ -259,6 +259,16 @@ veda_status veda_tile_map_maxpool(const veda_problem* p, const void* qp, const v
                                   const int32_t* rows, int32_t R, float scale, float* map,
                                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* veda_tile_map_maxpool on grid-order tensors: q, k [B, heads, N, d] bf16
+ * (read), no tile-major copies needed.  Each tile is fetched as one 5D box of
+ * the grid-order tensor, which holds the same values as the permuted tile
+ * (zeros in pad slots), so the map is identical to veda_tile_map_maxpool's on
+ * the permuted tensors.  Other arguments, workspace (veda_tile_map_workspace)
+ * and errors as for veda_tile_map_maxpool. */
+veda_status veda_tile_map_maxpool_grid(const veda_problem* p, const void* q, const void* k,
+                                       const int32_t* rows, int32_t R, float scale, float* map,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------------------- training the estimator */
 
 /* Bytes of workspace veda_distill_loss_grad needs. */

@@ -116,6 +116,9 @@ def test_peak_follows_the_clock_record():
     # below the maximum with no reason recorded: the burst figure still applies
     low = dict(at_max, sm_mhz=1852.0)
     assert bench.choose_peak(peaks, low, "measured")[0] == 1674.3
+    # the power cap flagged while the clock stays at its maximum: still burst
+    flagged = dict(at_max, reasons=["sw_power_cap"])
+    assert bench.choose_peak(peaks, flagged, "measured")[0] == 1674.3
 
 
 def test_loglog_slope():

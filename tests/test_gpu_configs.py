@@ -191,8 +191,9 @@ def test_attention_wan14b_dense_sampled(V):
 # ------------------------------------------------------------------ tile map at full size
 def test_tile_map_wan14b_sampled_rows(V):
     """The max-pooled full-attention map over 10% of the Q tiles at the
-    Wan2.1-14B shape (the distillation target's launch); sampled subset rows
-    of three heads against the oracle's explicit softmax rows."""
+    Wan2.1-14B shape (the distillation target's launch), from the permuted
+    copies and from grid order (identical maps); sampled subset rows of three
+    heads against the oracle's explicit softmax rows."""
     w = PRESETS["wan14b"]
     p = _problem(V, w)
     q, k, _ = cached_qkv(w, 0)
@@ -206,8 +207,12 @@ def test_tile_map_wan14b_sampled_rows(V):
     ws = torch.empty(V.veda_tile_map_workspace(p, R) // 4 + 64, dtype=torch.float32, device="cuda")
     mp = torch.full((p.B, p.heads, R, p.nt_max), float("nan"), dtype=torch.float32, device="cuda")
     V.veda_tile_map_maxpool(p, qp, kp, rows.cuda(), mp, ws)
+    # the grid-order entry point on the unpermuted tensors gives the same map
+    mg = torch.full_like(mp, float("nan"))
+    V.veda_tile_map_maxpool_grid(p, q.cuda(), k.cuda(), rows.cuda(), mg, ws)
     V.veda_sync_status()
-    del ws
+    assert torch.equal(mg, mp)
+    del ws, mg
     grid = (w.T, w.H, w.W)
     rng = np.random.default_rng(3)
     g = f64(mp)

@@ -113,6 +113,31 @@ def test_grid_attention_without_lse(V, gr):
     assert torch.equal(o, gr.out_g)
 
 
+def test_grid_tile_map_equals_tile_layout_and_oracle(V, gr):
+    """veda_tile_map_maxpool_grid on the grid-order tensors gives the same map,
+    bit for bit, as veda_tile_map_maxpool on the permuted copies (the tile
+    boxes hold the same values), and matches the oracle; the ten-tiling case
+    takes two pass-1 launches."""
+    from parity import MAP_REL
+    from veda_synth import make_map_rows
+    w, p = gr.w, gr.p
+    rows = make_map_rows(p.nt_per_head, w.B, 0.3, seed=2)
+    rows[0, -1] = -1  # an unused slot
+    R = rows.shape[1]
+    ws = torch.empty(V.veda_tile_map_workspace(p, R) // 4 + 64, dtype=torch.float32, device="cuda")
+    m_tile = torch.full((p.B, p.heads, R, p.nt_max), float("nan"), dtype=torch.float32, device="cuda")
+    m_grid = torch.full_like(m_tile, float("nan"))
+    V.veda_tile_map_maxpool(p, gr.tile.qp, gr.tile.kp, rows.cuda(), m_tile, ws)
+    V.veda_tile_map_maxpool_grid(p, gr.qd, gr.kd, rows.cuda(), m_grid, ws)
+    V.veda_sync_status()
+    assert torch.equal(m_grid, m_tile)
+    ref = O.tile_map_maxpool(gr.ora["qp"], gr.ora["kp"], rows.numpy(), gr.grid, w.tilings, w.S)
+    g = f64(m_grid)
+    big = ref >= 1e-8
+    assert np.all(np.abs(g[big] - ref[big]) <= MAP_REL * ref[big])
+    assert np.all(np.abs(g[~big] - ref[~big]) <= 1e-11)
+
+
 def test_grid_wan14b_full_size_sampled(V):
     """The benchmarked 14B shape in the grid layout, the launch the bench times: sampled Q tiles of
     sampled heads against the oracle, and the whole output equal to the tile-major path."""

@@ -75,6 +75,7 @@ _SIG = {
     "veda_attn_config": [_P, ctypes.c_int32, _I32P, _I32P, ctypes.POINTER(ctypes.c_size_t)],
     "veda_tile_map_workspace": [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)],
     "veda_tile_map_maxpool": [_P, _V, _V, _V, ctypes.c_int32, ctypes.c_float, _V, _V, ctypes.c_size_t, _V],
+    "veda_tile_map_maxpool_grid": [_P, _V, _V, _V, ctypes.c_int32, ctypes.c_float, _V, _V, ctypes.c_size_t, _V],
     "veda_distill_workspace": [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)],
     "veda_distill_loss_grad": [_P, _V, _V, ctypes.POINTER(veda_mlp), ctypes.POINTER(veda_mlp), _V, _V, ctypes.c_int32,
                                _V, ctypes.POINTER(veda_mlp_grad), ctypes.POINTER(veda_mlp_grad), _V, ctypes.c_size_t,
@@ -338,6 +339,19 @@ def veda_tile_map_maxpool(p: Problem, qp: torch.Tensor, kp: torch.Tensor, rows: 
         _ptr(rows, "rows", torch.int32, (p.B * p.heads, R)), R, ctypes.c_float(scale),
         _ptr(out, "map", torch.float32, (p.B, p.heads, R, p.nt_max)), _ptr(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream)), "veda_tile_map_maxpool")
+    return out
+
+
+def veda_tile_map_maxpool_grid(p: Problem, q: torch.Tensor, k: torch.Tensor, rows: torch.Tensor, out: torch.Tensor,
+                               workspace: torch.Tensor, scale: float = 0.0, stream=None) -> torch.Tensor:
+    """The max-pooled tile map from grid-order q, k [B, heads, N, d] bf16 (no tile-major copies)."""
+    gs = p.grid_shape()
+    R = int(rows.shape[-1])
+    _check(LIB.veda_tile_map_maxpool_grid(
+        p.ref, _ptr(q, "q", torch.bfloat16, gs), _ptr(k, "k", torch.bfloat16, gs),
+        _ptr(rows, "rows", torch.int32, (p.B * p.heads, R)), R, ctypes.c_float(scale),
+        _ptr(out, "map", torch.float32, (p.B, p.heads, R, p.nt_max)), _ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "veda_tile_map_maxpool_grid")
     return out
 
 

@@ -82,6 +82,11 @@ struct MapArgs {
   float* lse2;          // scratch [B*heads, R, S]          (log2 domain)
   float* map;           // [B, heads, R, NT_max]
   uint64_t timeout_ns;
+  // Grid-order pass-1 launches only: the heads this launch covers and, per
+  // head, which of the launch's tensor maps holds its tile box.
+  int32_t n_group;
+  int16_t head_list[VEDA_MAX_HEADS];
+  int8_t map_of_head[VEDA_MAX_HEADS];
 };
 
 cudaError_t launch_permute(const Geometry& G, const void* x, void* xp, cudaStream_t s, int sms);
@@ -111,6 +116,11 @@ cudaError_t launch_tripool_grid(const Geometry& G, const void* x, float* desc, c
 
 cudaError_t launch_tile_map(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,
                             const MapArgs& a, cudaStream_t s);
+// Grid-order tile map: pass 1 once per group of up to kMaxGridMaps distinct
+// tilings (a.head_list / a.map_of_head), then pass 2 once for all heads.
+cudaError_t launch_tile_map_pass1_grid(const Geometry& G, const AttnMaps<kMaxGridMaps>& m, const MapArgs& a,
+                                       cudaStream_t s);
+cudaError_t launch_tile_map_pass2(const Geometry& G, const MapArgs& a, cudaStream_t s);
 
 size_t distill_ws_bytes(const Geometry& G, int hidden, int e, int R);
 cudaError_t launch_head_error(const Geometry& G, const void* o, const void* o_ref, float* err, float* ref,

@@ -68,18 +68,44 @@ __device__ __forceinline__ bool map_warp_wait(uint32_t bar, uint32_t parity, vol
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int D, int BN>
+// GRID = false: Q and K are tile-major [B, heads, NT_max*S, d], a tile is a 2D
+// box of S rows.  GRID = true: Q and K stay in grid order [B, heads, N, d]; a
+// tile is the 5D box of its pt x ph x pw tokens, which lands in shared memory
+// in slot order with zeros for the parts outside the grid -- the same tile
+// contents the permutation writes -- so both layouts give identical maps.  A
+// grid-order launch covers the heads A.head_list[0 .. A.n_group), head h
+// using tensor maps number A.map_of_head[h].
+template <int D, int BN, bool GRID>
 __global__ void __launch_bounds__(320, 1)
-    tile_map_pass1_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+    tile_map_pass1_kernel(const __grid_constant__ AttnMaps<GRID ? kMaxGridMaps : 1> M,
                           const __grid_constant__ Geometry G, const __grid_constant__ MapArgs A) {
   using C = MapCfg<D, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = blockIdx.x % A.R;
-  const int bh = blockIdx.x / A.R;
-  const int h = bh % G.heads;
+  int bh, h, mi = 0;
+  if constexpr (GRID) {
+    const int hb = blockIdx.x / A.R;        // b * n_group + position in the head list
+    h = A.head_list[hb % A.n_group];
+    bh = (hb / A.n_group) * G.heads + h;
+    mi = A.map_of_head[h];
+  } else {
+    bh = blockIdx.x / A.R;
+    h = bh % G.heads;
+  }
   const HeadGeom hg = G.g[h];
+  const CUtensorMap* tmQ = &M.q[mi];
+  const CUtensorMap* tmK = &M.k[mi];
+  // Channel chunk c (64 channels) of tile j of this head into shared memory.
+  auto load_tile = [&](uint32_t dst, const CUtensorMap* map, uint32_t b, int c, int j) {
+    if constexpr (GRID) {
+      const int jw = j % hg.nTw, jh = (j / hg.nTw) % hg.nTh, jt = j / (hg.nTw * hg.nTh);
+      tma_load_5d(dst, map, b, 64 * c, jw * hg.pw, jh * hg.ph, jt * hg.pt, bh);
+    } else {
+      tma_load_2d(dst, map, b, 64 * c, (bh * G.ntmax + j) * G.S);
+    }
+  };
   const int i = A.rows[(long long)bh * A.R + r];
   if (i < 0 || i >= hg.nt) return;  // CTA-uniform
   const int S = G.S;
@@ -127,11 +153,11 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 0) {
     int issued = 0;
     if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(tmQ);
+      tma_prefetch_desc(tmK);
       mbar_arrive_expect_tx(bar(MBAR_Q), (uint32_t)(S * D * 2));
       for (int c = 0; c < D / 64; ++c)
-        tma_load_2d(sQ + c * C::kChunk, &tmQ, bar(MBAR_Q), 64 * c, (bh * G.ntmax + i) * S);
+        load_tile(sQ + c * C::kChunk, tmQ, bar(MBAR_Q), c, i);
     }
     for (int t = 0; t < nt; ++t) {
       const int st = t % C::kStages;
@@ -140,8 +166,7 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0 && VEDA_IN_BOUNDS(t < hg.nt && (long long)(bh * G.ntmax + t) * S < (long long)G.B * G.heads * G.ntmax * S)) {
         mbar_arrive_expect_tx(bar(MBAR_KFULL + st), (uint32_t)C::kKBytes);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_2d(sK + st * C::kKBytes + c * BN * 128, &tmK, bar(MBAR_KFULL + st), 64 * c,
-                      (bh * G.ntmax + t) * S);
+          load_tile(sK + st * C::kKBytes + c * BN * 128, tmK, bar(MBAR_KFULL + st), c, t);
       }
       __syncwarp();
       issued = t + 1;
@@ -327,32 +352,49 @@ __global__ void __launch_bounds__(256) tile_map_pass2_kernel(const __grid_consta
   }
 }
 
-template <int D, int BN>
-static cudaError_t launch_map_t(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,
-                                const MapArgs& a, cudaStream_t s) {
+template <int D, int BN, bool GRID>
+static cudaError_t launch_map_t(const Geometry& G, const AttnMaps<GRID ? kMaxGridMaps : 1>& m, const MapArgs& a,
+                                cudaStream_t s) {
   using C = MapCfg<D, BN>;
-  cudaError_t err = cudaFuncSetAttribute(tile_map_pass1_kernel<D, BN>,
+  cudaError_t err = cudaFuncSetAttribute(tile_map_pass1_kernel<D, BN, GRID>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
   if (err != cudaSuccess) return err;
-  const unsigned blocks = (unsigned)(G.B * G.heads * a.R);
-  tile_map_pass1_kernel<D, BN><<<blocks, C::kThreads, C::kSmem, s>>>(tq, tk, G, a);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  return cudaSuccess;
+  const unsigned blocks = (unsigned)(G.B * (GRID ? a.n_group : G.heads) * a.R);
+  tile_map_pass1_kernel<D, BN, GRID><<<blocks, C::kThreads, C::kSmem, s>>>(m, G, a);
+  return cudaGetLastError();
 }
 
-cudaError_t launch_tile_map(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,
-                            const MapArgs& a, cudaStream_t s) {
-  cudaError_t err;
-  if (G.d == 128 && G.S == 128) err = launch_map_t<128, 128>(G, tq, tk, a, s);
-  else if (G.d == 128 && G.S == 64) err = launch_map_t<128, 64>(G, tq, tk, a, s);
-  else if (G.d == 64 && G.S == 128) err = launch_map_t<64, 128>(G, tq, tk, a, s);
-  else err = launch_map_t<64, 64>(G, tq, tk, a, s);
-  if (err != cudaSuccess) return err;
+template <bool GRID>
+static cudaError_t launch_pass1(const Geometry& G, const AttnMaps<GRID ? kMaxGridMaps : 1>& m, const MapArgs& a,
+                                cudaStream_t s) {
+  if (G.d == 128 && G.S == 128) return launch_map_t<128, 128, GRID>(G, m, a, s);
+  if (G.d == 128 && G.S == 64) return launch_map_t<128, 64, GRID>(G, m, a, s);
+  if (G.d == 64 && G.S == 128) return launch_map_t<64, 128, GRID>(G, m, a, s);
+  return launch_map_t<64, 64, GRID>(G, m, a, s);
+}
+
+cudaError_t launch_tile_map_pass1_grid(const Geometry& G, const AttnMaps<kMaxGridMaps>& m, const MapArgs& a,
+                                       cudaStream_t s) {
+  return launch_pass1<true>(G, m, a, s);
+}
+
+cudaError_t launch_tile_map_pass2(const Geometry& G, const MapArgs& a, cudaStream_t s) {
   const long long total_threads = (long long)G.B * G.heads * a.R * G.ntmax * 32;
   long long blocks = (total_threads + 255) / 256;
   if (blocks > 148LL * 32) blocks = 148LL * 32;
   tile_map_pass2_kernel<<<(unsigned)blocks, 256, 0, s>>>(G, a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_tile_map(const Geometry& G, const CUtensorMap& tq, const CUtensorMap& tk,
+                            const MapArgs& a, cudaStream_t s) {
+  AttnMaps<1> m;
+  m.q[0] = tq;
+  m.k[0] = tk;
+  m.v[0] = tk;   // unused
+  cudaError_t err = launch_pass1<false>(G, m, a, s);
+  if (err != cudaSuccess) return err;
+  return launch_tile_map_pass2(G, a, s);
 }
 
 // A kernel whose only job is to run one bounded wait out: it waits on an

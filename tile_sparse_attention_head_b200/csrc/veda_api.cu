@@ -594,6 +594,7 @@ veda_status veda_tile_map_maxpool(const veda_problem* p, const void* qp, const v
   CUtensorMap tq, tk;
   if ((s = encode_tile_major(G, qp, &tq)) != VEDA_OK || (s = encode_tile_major(G, kp, &tk)) != VEDA_OK) return s;
   MapArgs a;
+  std::memset(&a, 0, sizeof(a));
   a.rows = rows;
   a.R = R;
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)G.d);
@@ -604,6 +605,70 @@ veda_status veda_tile_map_maxpool(const veda_problem* p, const void* qp, const v
   a.timeout_ns = g_timeout_ns;
   cudaError_t e = launch_tile_map(G, tq, tk, a, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "veda_tile_map_maxpool");
+  return ok();
+}
+
+veda_status veda_tile_map_maxpool_grid(const veda_problem* p, const void* q, const void* k, const int32_t* rows,
+                                       int32_t R, float scale, float* map, void* workspace, size_t workspace_bytes,
+                                       void* stream) {
+  Geometry G;
+  veda_status s = make_geometry(p, &G);
+  if (s != VEDA_OK) return s;
+  if (R < 1) return fail(VEDA_ERR_INVALID_ARG, "R must be >= 1 (got %d)", R);
+  if (!q || !k || !rows || !map || !workspace) return fail(VEDA_ERR_INVALID_ARG, "NULL tensor argument");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(map) || !aligned16(rows))
+    return fail(VEDA_ERR_INVALID_ARG, "tensor arguments must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(VEDA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (workspace_bytes < map_ws_bytes(G, R))
+    return fail(VEDA_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, map_ws_bytes(G, R));
+  if ((long long)G.B * G.heads * R >= (1LL << 31)) return fail(VEDA_ERR_INVALID_ARG, "B*heads*R too large");
+  if (!(std::isfinite(scale))) return fail(VEDA_ERR_INVALID_ARG, "scale must be finite");
+  // Distinct tilings in order of first appearance; one pass-1 launch covers up
+  // to kMaxGridMaps of them (one set of tensor maps each).
+  int tiling_of_head[VEDA_MAX_HEADS];
+  int distinct[VEDA_MAX_HEADS];
+  int n_distinct = 0;
+  for (int h = 0; h < G.heads; ++h) {
+    int u = 0;
+    while (u < n_distinct && !(G.g[distinct[u]].pt == G.g[h].pt && G.g[distinct[u]].ph == G.g[h].ph &&
+                               G.g[distinct[u]].pw == G.g[h].pw))
+      ++u;
+    if (u == n_distinct) distinct[n_distinct++] = h;
+    tiling_of_head[h] = u;
+  }
+  MapArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.rows = rows;
+  a.R = R;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)G.d);
+  a.scale_log2 = sc * 1.4426950408889634f;
+  a.rowmax = static_cast<float*>(workspace);
+  a.lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + map_rowmax_bytes(G, R));
+  a.map = map;
+  a.timeout_ns = g_timeout_ns;
+  AttnMaps<kMaxGridMaps> maps;  // copied into the kernel parameters at launch
+  std::memset(&maps, 0, sizeof(maps));
+  for (int u0 = 0; u0 < n_distinct; u0 += kMaxGridMaps) {
+    const int nu = std::min(kMaxGridMaps, n_distinct - u0);
+    for (int u = 0; u < nu; ++u) {
+      const HeadGeom& hg = G.g[distinct[u0 + u]];
+      if ((s = encode_grid_tiles(G, q, hg, &maps.q[u])) != VEDA_OK ||
+          (s = encode_grid_tiles(G, k, hg, &maps.k[u])) != VEDA_OK)
+        return s;
+      maps.v[u] = maps.k[u];   // unused by the map
+    }
+    a.n_group = 0;
+    for (int h = 0; h < G.heads; ++h) {
+      const int u = tiling_of_head[h] - u0;
+      if (u < 0 || u >= nu) continue;
+      a.head_list[a.n_group++] = (int16_t)h;
+      a.map_of_head[h] = (int8_t)u;
+    }
+    cudaError_t e = launch_tile_map_pass1_grid(G, maps, a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "veda_tile_map_maxpool_grid (pass 1)");
+  }
+  cudaError_t e = launch_tile_map_pass2(G, a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "veda_tile_map_maxpool_grid (pass 2)");
   return ok();
 }
 
