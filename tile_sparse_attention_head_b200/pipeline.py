@@ -152,7 +152,7 @@ class VedaAttentionHost:
     layout); the copies are cudaMemcpyAsync from pinned memory.
     """
 
-    def __init__(self, problem: B.Problem, mlp_q, mlp_k, keep_ratio: float, device="cuda", chunk_heads: int = 5,
+    def __init__(self, problem: B.Problem, mlp_q, mlp_k, keep_ratio: float, device="cuda", chunk_heads: int = 2,
                  slots: int = 3):
         p = problem
         self.p = p
