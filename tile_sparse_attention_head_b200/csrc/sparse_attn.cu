@@ -197,7 +197,11 @@ __device__ __forceinline__ int next_attn_item(const Geometry& G, const AttnArgs&
 __device__ __forceinline__ uint32_t div_by_recip(uint32_t j, uint64_t m) {
   return (uint32_t)(((uint64_t)j * m) >> 32);
 }
-__device__ __forceinline__ uint64_t recip_ceil(uint32_t n) { return (0x100000000ull + n - 1) / n; }
+// ceil(2^32 / n) from a 32-bit division: floor((2^32 - 1) / n) + 1 for n >= 2
+// (equal whether or not n divides 2^32), 2^32 for n = 1.
+__device__ __forceinline__ uint64_t recip_ceil(uint32_t n) {
+  return n == 1u ? 0x100000000ull : (uint64_t)(0xffffffffu / n) + 1ull;
+}
 
 // GRID = false: Q/K/V/O are tile-major [B, heads, NT_max*S, d]; tile j of a
 // head is rows j*S .. j*S+S-1, fetched as one 2D box per 64 channels.
@@ -225,10 +229,14 @@ __global__ void __launch_bounds__(384, 1)
   const int cap = C::list_cap(A.k_max);
   const int n_items = G.B * (GRID ? A.n_group : G.heads) * G.ntmax;
   // Channel chunk c (64 channels) of tile j of head row bh into shared memory at dst.
-  auto load_tile = [&](uint32_t dst, const CUtensorMap* map, uint32_t b, int c, const HeadGeom& hg, int bh, int j) {
+  auto load_tile = [&](uint32_t dst, const CUtensorMap* map, uint32_t b, int c, const HeadGeom& hg, int bh, int j,
+                       uint64_t r_w, uint64_t r_h) {
     if constexpr (GRID) {
-      const int jw = j % hg.nTw, jh = (j / hg.nTw) % hg.nTh, jt = j / (hg.nTw * hg.nTh);
-      tma_load_5d(dst, map, b, 64 * c, jw * hg.pw, jh * hg.ph, jt * hg.pt, bh);
+      // tile coordinates from exact reciprocals of the head's tile counts
+      const uint32_t jq = div_by_recip((uint32_t)j, r_w);
+      const uint32_t jt = div_by_recip(jq, r_h);
+      const int jw = j - (int)jq * hg.nTw, jh = (int)jq - (int)jt * hg.nTh;
+      tma_load_5d(dst, map, b, 64 * c, jw * hg.pw, jh * hg.ph, (int)jt * hg.pt, bh);
     } else {
       tma_load_2d(dst, map, b, 64 * c, (bh * G.ntmax + j) * S);
     }
@@ -332,7 +340,8 @@ __global__ void __launch_bounds__(384, 1)
         tma_prefetch_desc(tmQ);
         tma_prefetch_desc(&M.k[x.mi]);
         mbar_arrive_expect_tx(bar(BAR_QFULL), (uint32_t)(S * D * 2));
-        for (int c = 0; c < D / 64; ++c) load_tile(sQ + c * C::kChunk, tmQ, bar(BAR_QFULL), c, hg, x.bh, x.i);
+        const uint64_t rw = recip_ceil((uint32_t)hg.nTw), rh = recip_ceil((uint32_t)hg.nTh);
+        for (int c = 0; c < D / 64; ++c) load_tile(sQ + c * C::kChunk, tmQ, bar(BAR_QFULL), c, hg, x.bh, x.i, rw, rh);
       }
       __syncwarp();
       ++q_fills;
@@ -345,6 +354,7 @@ __global__ void __launch_bounds__(384, 1)
       const int slot = n & 1;
       const HeadGeom hg = G.g[it.h];
       const CUtensorMap* tmK = &M.k[it.mi];
+      const uint64_t rw = recip_ceil((uint32_t)hg.nTw), rh = recip_ceil((uint32_t)hg.nTh);
       __syncwarp();   // this warp's own list writes are visible to lane 0
       const int nsel = misc[4 + slot];
       AttnItem nx;
@@ -363,7 +373,7 @@ __global__ void __launch_bounds__(384, 1)
           if (VEDA_IN_BOUNDS(j >= 0 && j < hg.nt)) {   // a skipped fetch runs the consumers' waits out
             mbar_arrive_expect_tx(bar(BAR_KFULL + st), (uint32_t)C::kTileBytes);
             for (int c = 0; c < D / 64; ++c)
-              load_tile(sK + st * C::kTileBytes + c * BN * 128, tmK, bar(BAR_KFULL + st), c, hg, it.bh, j);
+              load_tile(sK + st * C::kTileBytes + c * BN * 128, tmK, bar(BAR_KFULL + st), c, hg, it.bh, j, rw, rh);
           }
         }
         __syncwarp();
@@ -398,6 +408,7 @@ __global__ void __launch_bounds__(384, 1)
       const int nsel = misc[4 + slot];
       const HeadGeom hg = G.g[it.h];
       const CUtensorMap* tmV = &M.v[it.mi];
+      const uint64_t rw = recip_ceil((uint32_t)hg.nTw), rh = recip_ceil((uint32_t)hg.nTh);
       if (lane == 0) tma_prefetch_desc(tmV);
       for (int t = 0; t < nsel; ++t, ++vt) {
         const int st = vt % VST, fill = vt / VST;
@@ -407,7 +418,7 @@ __global__ void __launch_bounds__(384, 1)
           if (VEDA_IN_BOUNDS(j >= 0 && j < hg.nt)) {
             mbar_arrive_expect_tx(bar(BAR_VFULL + st), (uint32_t)C::kTileBytes);
             for (int c = 0; c < D / 64; ++c)
-              load_tile(sV + st * C::kTileBytes + c * BN * 128, tmV, bar(BAR_VFULL + st), c, hg, it.bh, j);
+              load_tile(sV + st * C::kTileBytes + c * BN * 128, tmV, bar(BAR_VFULL + st), c, hg, it.bh, j, rw, rh);
           }
         }
         __syncwarp();
