@@ -56,7 +56,7 @@ WORKLOAD_NAMES = {"wan14b": "Wan2.1-14B-720p-81f 21x45x80 (75,600 tokens) 40 hea
 # keyed by workload and layout and tied to the kernel source it was measured
 # on: reported only while csrc/sparse_attn.cu still hashes to that version.
 ATTN_TRAFFIC = {("wan14b", "tile"): {"bytes": 1.26e9 + 858.49e6, "src_sha256_16": "b5a8f826b6c7f91f"},
-                ("wan14b", "grid"): {"bytes": 1139.32e6 + 740.37e6, "src_sha256_16": "1805a41c0b164c3f"}}
+                ("wan14b", "grid"): {"bytes": 1139.90e6 + 740.74e6, "src_sha256_16": "6768221b7d236b48"}}
 
 
 def attn_traffic(workload: str, layout: str):
