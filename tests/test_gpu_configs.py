@@ -3,6 +3,10 @@
 The launch picks kernel variants from the problem size, and the benchmark
 workloads reach variants that the small parity cases do not:
 
+* top-k over rows of 257-512, 513-768 and 769-1,024 tiles: the register
+  bisection with 16, 24 and 32 keys per lane (the Wan2.1-1.3B shape has up to
+  336 tiles per head, the Wan2.1-14B shape 720), with every feature width the
+  score kernel stages (e = 16, 32, 64, 128);
 * top-k over rows of 1,025-2,048 tiles: the register bisection with 64 keys
   per lane (the 245,760-token sweep has 1,920 tiles per head);
 * top-k over rows of more than 2,048 tiles: the radix select;
@@ -85,6 +89,14 @@ def _check_selection(V, w, att, ora, heads, check_probs):
 # Two heads of unequal tile counts each, so the launch covers rows of both
 # lengths and rows past a head's own count.
 TOPK_CASES = [
+    # 330 and 360 tiles: 16 keys per lane, e = 16
+    wl("topk360", (12, 40, 44), 1, 2, 64, 64, [(4, 4, 4), (1, 8, 8)], 0.05, 128, 16, "rff"),
+    # 660 and 720 tiles: 24 keys per lane (as in the Wan2.1-14B launch), e = 32
+    wl("topk720", (24, 40, 44), 1, 2, 64, 64, [(4, 4, 4), (2, 4, 8)], 0.05, 128, 32, "rff"),
+    # 600 tiles, e = 128: phi_k staged partly from registers, partly directly
+    wl("topk600e128", (24, 40, 40), 1, 1, 64, 64, [(4, 4, 4)], 0.05, 128, 128, "rff"),
+    # 770 and 715 tiles at d = 128: 32 keys per lane, e = 64
+    wl("topk770", (26, 42, 40), 1, 2, 128, 64, [(4, 4, 4), (2, 4, 8)], 0.05, 256, 64, "rff"),
     # 1,650 tiles: the 64-keys-per-lane register bisection
     wl("topk1650", (39, 41, 58), 1, 2, 64, 64, [(4, 4, 4), (2, 4, 8)], 0.05, 128, 32, "rff"),
     # 2,145 and 2,200 tiles: the radix select
@@ -95,9 +107,9 @@ TOPK_CASES = [
 
 
 @pytest.mark.parametrize("w", TOPK_CASES, ids=[w.name for w in TOPK_CASES])
-def test_topk_long_rows_against_oracle(V, w):
+def test_topk_row_lengths_against_oracle(V, w):
     p = _problem(V, w)
-    assert p.nt_max > 1024
+    assert p.nt_max > 256
     q, k, _ = make_qkv(w, seed=0)
     m = make_mlp(w, seed=1)
     att = _select_on_gpu(V, w, q, k, m, want_probs=True)

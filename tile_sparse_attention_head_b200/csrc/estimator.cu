@@ -124,26 +124,38 @@ __global__ void __launch_bounds__(kEstThreads, 1)
     const int n1 = min(kEstN1, hidden - n0);
     const int n1p = (n1 + 15) & ~15;
     // ------------------------------------------------------------ layer 1
+    // A panel: 128 descriptor rows x 32 features; B panel: up to 256 W1 rows
+    // (hidden units n0 ..) x 32 features.  16-byte piece t of a panel is row
+    // t / 8, chunk t % 8, and thread tid takes pieces tid + 256 q, so a warp
+    // reads four whole 128-byte row segments per load.  Panel kc + 1 is
+    // loaded into registers as soon as panel kc is stored, so its load
+    // latency overlaps the barrier and the products of panel kc.
+    const int pr = tid >> 3, pc = tid & 7;   // row and chunk of piece tid
+    float4 xv[4], wv[8];
+    auto load_panel = [&](int kc) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int r = pr + 32 * q;
+        xv[q] = (r < nrows) ? __ldg(reinterpret_cast<const float4*>(X + (long long)r * K1 + kc * 32) + pc)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int r = pr + 32 * q;
+        wv[q] = (r < n1) ? __ldg(reinterpret_cast<const float4*>(W1 + (long long)(n0 + r) * K1 + kc * 32) + pc)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    load_panel(0);
     for (int kc = 0; kc < K1 / 32; ++kc) {
-      // descriptor panel: thread -> row tid/2, chunks 4*(tid&1) .. +3
-      // W1 panel: thread -> hidden unit n0 + tid, all 8 chunks
-      float4 xv[4], wv[8];
-      const int xr = tid >> 1, xc = (tid & 1) * 4;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        xv[q] = (xr < nrows) ? __ldg(reinterpret_cast<const float4*>(X + (long long)xr * K1 + kc * 32) + xc + q)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        wv[q] = (tid < n1) ? __ldg(reinterpret_cast<const float4*>(W1 + (long long)(n0 + tid) * K1 + kc * 32) + q)
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
       ok = wait_stage(use) && ok;
       uint8_t* st = stage(use);
       uint8_t *ahi = st, *alo = st + kEstPanelA, *bhi = st + 2 * kEstPanelA, *blo = bhi + kEstPanelB;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) store_split4(ahi, alo, xr, xc + q, xv[q]);
+      for (int q = 0; q < 4; ++q) store_split4(ahi, alo, pr + 32 * q, pc, xv[q]);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) store_split4(bhi, blo, tid, q, wv[q]);
+      for (int q = 0; q < 8; ++q) store_split4(bhi, blo, pr + 32 * q, pc, wv[q]);
+      if (kc + 1 < K1 / 32) load_panel(kc + 1);
       fence_proxy_async_smem();
       tc_fence_before();
       ok = __syncthreads_and(ok);
@@ -173,6 +185,21 @@ __global__ void __launch_bounds__(kEstThreads, 1)
     ok = __syncthreads_and(ok);
     if (!ok) break;
     // ------------------------------------------------------------ layer 2
+    // W2[o, u0 .. u0+31] for every output o, staged by warps 4-7: thread
+    // t = tid - 128 takes 16-byte chunks t, t + 128, ... (E * 8 of them); the
+    // next panel's chunks are loaded while the current one is multiplied.
+    constexpr int kW2Per = (E * 8 + 127) / 128;
+    float4 w2v[kW2Per];
+    auto load_w2 = [&](int u0) {
+#pragma unroll
+      for (int q = 0; q < kW2Per; ++q) {
+        const int t = tid - 128 + q * 128;
+        const int o = t >> 3, unit = u0 + (t & 7) * 4;
+        w2v[q] = (t < E * 8 && unit < hidden) ? __ldg(reinterpret_cast<const float4*>(W2 + (long long)o * hidden + unit))
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    if (warp >= 4) load_w2(n0);
     for (int pi = 0; pi < (n1 + 31) / 32; ++pi) {
       const int u0 = n0 + pi * 32;   // first hidden unit of this panel
       ok = wait_stage(use) && ok;
@@ -201,14 +228,12 @@ __global__ void __launch_bounds__(kEstThreads, 1)
           store_split4(ahi, alo, r, c, hv);
         }
       } else {
-        // W2[o, u0 .. u0+31] for every output o
-        for (int t = tid - 128; t < E * 8; t += 128) {
-          const int o = t >> 3, c = t & 7;
-          const int unit = u0 + c * 4;
-          const float4 wv = (unit < hidden) ? __ldg(reinterpret_cast<const float4*>(W2 + (long long)o * hidden + unit))
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
-          store_split4(bhi, blo, o, c, wv);
+#pragma unroll
+        for (int q = 0; q < kW2Per; ++q) {
+          const int t = tid - 128 + q * 128;
+          if (t < E * 8) store_split4(bhi, blo, t >> 3, t & 7, w2v[q]);
         }
+        if (pi + 1 < (n1 + 31) / 32) load_w2(u0 + 32);
       }
       fence_proxy_async_smem();
       tc_fence_before();

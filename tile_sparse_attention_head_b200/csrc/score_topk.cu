@@ -7,8 +7,8 @@
 //   estimator_kernel  phi = W2 relu(W1 desc + b1) + b2 for every Q and K tile,
 //                     on the tensor cores at fp32 accuracy (estimator.cu),
 //                     written to the workspace;
-//   score_topk_kernel (score_topk_tc_kernel for rows of more than 1,024
-//                     tiles, scores on the tensor cores)
+//   score_topk_tc_kernel (scores on the tensor cores; feature widths e up
+//                     to 64) or score_topk_kernel (fp32 SIMT scores, e = 128)
 //                     per block of Q-tile rows: s = phi_q phi_k^T / sqrt(e)
 //                     into shared memory, optional row softmax, then the
 //                     exact k-th largest score per row and an ascending
@@ -89,12 +89,12 @@ constexpr int kQRows = 16;         // most Q-tile rows per CTA (the score tile i
 // Optional row softmax and the exact top-k of a block of Q-tile rows whose
 // scores s_scores [qb][ntpad] are in shared memory (rows i0 .. i0+qb-1 of
 // head row bh; nrows of them exist).  One warp per row.
-template <int KPL>
+template <int KPL, int NWARPS>
 __device__ __forceinline__ void select_rows(const Geometry& G, const TopkArgs& args, const float* s_scores,
                                             uint32_t* s_hist, int qb, int ntpad, int nrows, int nt, int k, int i0,
                                             int32_t* idx_base, float* probs_base, int warp, int lane) {
   uint32_t* hist = s_hist + warp * 256;
-  for (int r = warp; r < qb; r += kScoreThreads / 32) {
+  for (int r = warp; r < qb; r += NWARPS) {
     const int i = i0 + r;
     if (i >= G.ntmax) break;
     int32_t* irow = idx_base + (long long)i * args.k_max;
@@ -134,6 +134,28 @@ __device__ __forceinline__ void select_rows(const Geometry& G, const TopkArgs& a
       int gt = 0;
       prefix = kth_key_bisect(key, nt, k, lane, &gt);
       remaining = k - gt;
+      // Every key above the k-th largest and the first `remaining` keys equal
+      // to it (smallest tile indices), in ascending column order; column
+      // i * 32 + lane is key[i] of this lane.
+      int out = 0, eq_taken = 0;
+#pragma unroll
+      for (int i = 0; i < (KPL > 0 ? KPL : 1); ++i) {
+        if (i * 32 >= nt) break;   // warp-uniform
+        const int c = i * 32 + lane;
+        const bool in = c < nt;
+        const bool gt_ = in && key[i] > prefix;
+        const bool eq = in && key[i] == prefix;
+        const unsigned eqmask = __ballot_sync(0xffffffffu, eq);
+        const int eq_before = __popc(eqmask & ((1u << lane) - 1u));
+        const bool take = gt_ || (eq && eq_taken + eq_before < remaining);
+        const unsigned tmask = __ballot_sync(0xffffffffu, take);
+        const int pos = out + __popc(tmask & ((1u << lane) - 1u));
+        if (take && pos < k && VEDA_IN_BOUNDS(c < nt && pos < args.k_max)) irow[pos] = c;
+        out += __popc(tmask);
+        eq_taken += __popc(eqmask);
+      }
+      for (int c = k + lane; c < args.k_max; c += 32) irow[c] = -1;
+      continue;
     } else {
     // Radix select: find the k-th largest key, 8 bits per pass from the top.
     uint32_t pmask = 0;
@@ -252,23 +274,49 @@ __global__ void __launch_bounds__(kScoreThreads)
   }
   const float inv_sqrt_e = rsqrtf((float)e);
 
-  // Scores, one 16 x 128 tile per chunk of K tiles.
+  // Scores, one 16 x 128 tile per chunk of K tiles.  phi_k rows jc .. jc+127
+  // are staged transposed; 16-byte piece t of the chunk is row t % 128,
+  // features 4 (t / 128) .. +3, so consecutive threads take consecutive rows
+  // and the transposed stores do not conflict.  The first kPf pieces of each
+  // thread (all of them for e <= 64) are loaded into registers while the
+  // previous chunk's scores are formed.
+  constexpr int kPf = kKChunk * 16 / kScoreThreads;
+  const int npiece = kKChunk * (e / 4);
+  float4 pf[kPf];
+  auto load_pf = [&](int jc) {
+    const int ncols = min(kKChunk, nt - jc);
+#pragma unroll
+    for (int q = 0; q < kPf; ++q) {
+      const int t = tid + q * kScoreThreads;
+      const int jj = t % kKChunk, q4 = t / kKChunk;
+      pf[q] = (t < npiece && jj < ncols) ? __ldg(reinterpret_cast<const float4*>(phk + (long long)(jc + jj) * e) + q4)
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto put = [&](int t, float4 v) {
+    const int jj = t % kKChunk, q4 = t / kKChunk;
+    s_phik[(4 * q4 + 0) * kKChunk + jj] = v.x;
+    s_phik[(4 * q4 + 1) * kKChunk + jj] = v.y;
+    s_phik[(4 * q4 + 2) * kKChunk + jj] = v.z;
+    s_phik[(4 * q4 + 3) * kKChunk + jj] = v.w;
+  };
+  load_pf(0);
   const int cg = tid & 31, rp = tid >> 5;
   for (int jc = 0; jc < nt; jc += kKChunk) {
     __syncthreads();
     const int ncols = min(kKChunk, nt - jc);
-    // phi_k rows jc .. jc+127, transposed; consecutive threads take
-    // consecutive rows, so the transposed stores do not conflict.
-    for (int t = tid; t < kKChunk * (e / 4); t += kScoreThreads) {
+#pragma unroll
+    for (int q = 0; q < kPf; ++q) {
+      const int t = tid + q * kScoreThreads;
+      if (t < npiece) put(t, pf[q]);
+    }
+    for (int t = tid + kPf * kScoreThreads; t < npiece; t += kScoreThreads) {   // e > 64 only
       const int jj = t % kKChunk, q4 = t / kKChunk;
-      const float4 v = (jj < ncols) ? __ldg(reinterpret_cast<const float4*>(phk + (long long)(jc + jj) * e) + q4)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-      s_phik[(4 * q4 + 0) * kKChunk + jj] = v.x;
-      s_phik[(4 * q4 + 1) * kKChunk + jj] = v.y;
-      s_phik[(4 * q4 + 2) * kKChunk + jj] = v.z;
-      s_phik[(4 * q4 + 3) * kKChunk + jj] = v.w;
+      put(t, (jj < ncols) ? __ldg(reinterpret_cast<const float4*>(phk + (long long)(jc + jj) * e) + q4)
+                          : make_float4(0.f, 0.f, 0.f, 0.f));
     }
     __syncthreads();
+    if (jc + kKChunk < nt) load_pf(jc + kKChunk);
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll 8
     for (int cc = 0; cc < e; ++cc) {
@@ -296,46 +344,62 @@ __global__ void __launch_bounds__(kScoreThreads)
   }
   __syncthreads();
 
-  select_rows<KPL>(G, args, s_scores, s_hist, qb, ntpad, nrows, nt, k, i0, idx_base, probs_base, warp, lane);
+  select_rows<KPL, kScoreThreads / 32>(G, args, s_scores, s_hist, qb, ntpad, nrows, nt, k, i0, idx_base, probs_base,
+                                       warp, lane);
 }
 
 // ---------------------------------------------------------------------------
-// Scores on the tensor cores.  Per chunk of 128 K tiles (the MMA's M) and the
-// CTA's block of up to 16 Q rows (N = 16): S^T = phi_k phi_q^T with
-// tcgen05.mma kind::tf32 at fp32 accuracy -- each operand split as x = hi + lo
-// (hi the nearest tf32 value) and each product formed as hi*hi + hi*lo +
-// lo*hi, about 2^-21 relative, the same split the estimator uses.  The
-// accumulator lands in TMEM with one K tile per lane; warps 0-3 scale it and
-// write the chunk's column of the shared score block, from which the same
-// row softmax and top-k as above select the tiles.  phi_k is staged split into
-// 128-byte-swizzled K-major panels; the next chunk's rows are loaded into
-// registers while the current chunk's products run.  Feature widths e up to
-// 64 (panels of 32 features; e = 16 is zero-padded to 32).
+// Scores on the tensor cores.  A CTA takes a block of up to 32 Q-tile rows of
+// one head (the MMA's N, 16 or 32) and walks the head's K tiles in chunks of
+// 128 (the MMA's M): S^T = phi_k phi_q^T with tcgen05.mma kind::tf32 at fp32
+// accuracy -- each operand split as x = hi + lo (hi the nearest tf32 value)
+// and each product formed as hi*hi + hi*lo + lo*hi, about 2^-21 relative,
+// the same split the estimator uses.
+//
+//   A operand: a 3-stage ring, one stage per 32-feature panel of a chunk
+//     (hi and lo, 128-byte-swizzled K-major).  Every thread stages 16-byte
+//     pieces of the panel (a warp reads four whole 128-byte row segments per
+//     load); the pieces of the next stage are loaded into registers while
+//     the current stage is stored and multiplied.
+//   B operand: the block's phi_q rows, split once.
+//   Accumulators: four 32-column TMEM buffers, chunk c in buffer c % 4.  The
+//     chunk's products are read back two chunks later by warps 0-7 (one K tile
+//     per lane, 16 Q rows per warp), so the products never wait for the read
+//     and the read never waits for the products.  The scores land in a shared
+//     block [rows][ntpad], from which the row softmax and top-k of the SIMT
+//     kernel select the tiles, one warp per row.
+// Waits are bounded; the whole CTA agrees on an abort at every barrier, and
+// every MMA completes before TMEM is released.
 // ---------------------------------------------------------------------------
-constexpr int kTcRows = 16;     // Q rows per CTA: the MMA's N
-constexpr int kTcCols = 128;    // K tiles per chunk: the MMA's M
+constexpr int kTcCols = 128;     // K tiles per chunk: the MMA's M
+constexpr int kTcMaxRows = 32;   // Q rows per CTA at most: the MMA's N
+constexpr int kTcStages = 3;     // A-operand ring depth (one 32-feature panel pair per stage)
+constexpr int kTcAcc = 4;        // TMEM accumulator buffers of 32 columns
 
 template <int KP>
 struct ScoreTcCfg {
   static constexpr int kPanels = KP / 32;
-  static constexpr int kAPanel = kTcCols * 128;   // 128 K-tile rows x 32 fp32
-  static constexpr int kBPanel = kTcRows * 128;   // 16 Q rows x 32 fp32
-  static constexpr int kOffAhi = 0;
-  static constexpr int kOffAlo = kPanels * kAPanel;
-  static constexpr int kOffBhi = 2 * kPanels * kAPanel;
+  static constexpr int kAPanel = kTcCols * 128;      // 128 K-tile rows x 32 fp32
+  static constexpr int kStage = 2 * kAPanel;         // hi, lo
+  static constexpr int kBPanel = kTcMaxRows * 128;   // 32 Q rows x 32 fp32
+  static constexpr int kOffA = 0;
+  static constexpr int kOffBhi = kTcStages * kStage;
   static constexpr int kOffBlo = kOffBhi + kPanels * kBPanel;
-  static constexpr int kOffBar = kOffBlo + kPanels * kBPanel;   // [0] products done, [1] drain; misc after
-  static constexpr int kOffScores = kOffBar + 64;
-  static size_t smem_bytes(int qb, int ntpad, bool radix) {
-    return 1024 + kOffScores + sizeof(float) * (size_t)qb * ntpad + (radix ? sizeof(uint32_t) * 8 * 256 : 0);
+  static constexpr int kOffBar = kOffBlo + kPanels * kBPanel;   // stage free [3], accumulator full [4], drain; misc
+  static constexpr int kOffScores = kOffBar + 128;
+  static size_t smem_bytes(int qb, int ntpad, bool radix, int nthreads) {
+    return 1024 + kOffScores + sizeof(float) * (size_t)qb * ntpad +
+           (radix ? sizeof(uint32_t) * (nthreads / 32) * 256 : 0);
   }
 };
 
-template <int KPL, int KP>
-__global__ void __launch_bounds__(kScoreThreads, 1)
+template <int KPL, int KP, int NTHR>
+__global__ void __launch_bounds__(NTHR, 1)
     score_topk_tc_kernel(const __grid_constant__ Geometry G, const float* __restrict__ phi, int e, int qb,
                          int ntpad, const __grid_constant__ TopkArgs args) {
   using C = ScoreTcCfg<KP>;
+  constexpr int kP = C::kPanels;
+  constexpr int kPieces = kTcCols * 8 / NTHR;   // 16-byte pieces of an A panel per thread
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int bh = blockIdx.y;
@@ -352,16 +416,18 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     for (int r = 0; r < qb; ++r) {
       const int i = i0 + r;
       if (i >= G.ntmax) break;
-      for (int c = tid; c < args.k_max; c += kScoreThreads) idx_base[(long long)i * args.k_max + c] = -1;
+      for (int c = tid; c < args.k_max; c += NTHR) idx_base[(long long)i * args.k_max + c] = -1;
       if (probs_base)
-        for (int c = tid; c < G.ntmax; c += kScoreThreads) probs_base[(long long)i * G.ntmax + c] = 0.f;
+        for (int c = tid; c < G.ntmax; c += NTHR) probs_base[(long long)i * G.ntmax + c] = 0.f;
     }
     return;   // CTA-uniform, before any barrier or TMEM use
   }
   const int nrows = min(qb, nt - i0);
-  uint8_t *ahi = smem + C::kOffAhi, *alo = smem + C::kOffAlo, *bhi = smem + C::kOffBhi, *blo = smem + C::kOffBlo;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  int* misc = reinterpret_cast<int*>(bars + 2);   // [0] TMEM base, [1] abort
+  const int nq = qb > 16 ? 32 : 16;   // the MMA's N
+  uint8_t* bhi = smem + C::kOffBhi;
+  uint8_t* blo = smem + C::kOffBlo;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);   // [0,3) stage free, [3,7) acc full, [7] drain
+  int* misc = reinterpret_cast<int*>(bars + 8);                         // [0] TMEM base, [1] abort
   float* s_scores = reinterpret_cast<float*>(smem + C::kOffScores);
   uint32_t* s_hist = reinterpret_cast<uint32_t*>(s_scores + (size_t)qb * ntpad);
   volatile int* abort = misc + 1;
@@ -369,113 +435,126 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   const float* phq = phi + ((long long)bh * G.ntmax + i0) * e;
   const float* phk = phi + (((long long)G.B * G.heads + bh) * G.ntmax) * e;
   if (tid == 0) {
-    mbar_init(smem_u32(&bars[0]), 1);
-    mbar_init(smem_u32(&bars[1]), 1);
+    for (int b = 0; b < 8; ++b) mbar_init(smem_u32(&bars[b]), 1);
     misc[1] = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(&misc[0]), 32);
+    tmem_alloc(smem_u32(&misc[0]), kTcAcc * 32);
     tmem_relinquish();
   }
-  // phi_q of the CTA's rows, split, as the B operand (rows past nrows and
-  // features past e are zero): one 16-byte chunk per thread and pass.
-  for (int t = tid; t < kTcRows * (KP / 4); t += kScoreThreads) {
+  // phi_q of the block's rows, split, as the B operand (rows past nrows and
+  // features past e are zero).
+  for (int t = tid; t < kTcMaxRows * (KP / 4); t += NTHR) {
     const int r = t / (KP / 4), c = t % (KP / 4);
     const float4 v = (r < nrows && 4 * c < e) ? __ldg(reinterpret_cast<const float4*>(phq + (long long)r * e) + c)
                                               : make_float4(0.f, 0.f, 0.f, 0.f);
     store_split4(bhi + (c >> 3) * C::kBPanel, blo + (c >> 3) * C::kBPanel, r, c & 7, v);
   }
-  // The chunk's phi_k rows: thread -> row tid/2, KP/8 consecutive 16-byte chunks.
-  const int lr = tid >> 1, lc0 = (tid & 1) * (KP / 8);
-  float4 xv[KP / 8];
-  auto load_chunk = [&](int jc) {
+  // Stage u is chunk u / kP, panel u % kP.  Piece tid + NTHR q of a panel is
+  // K-tile row (tid + NTHR q) / 8, 16-byte chunk tid % 8.
+  const int nch = (nt + kTcCols - 1) / kTcCols;
+  const int nst = nch * kP;
+  const int pc = tid & 7;
+  float4 xv[kPieces];
+  auto load_stage = [&](int u) {
+    const int jc = (u / kP) * kTcCols, f0 = (u % kP) * 32 + 4 * pc;
 #pragma unroll
-    for (int q = 0; q < KP / 8; ++q) {
-      const int c = lc0 + q;
-      xv[q] = (jc + lr < nt && 4 * c < e)
-                  ? __ldg(reinterpret_cast<const float4*>(phk + (long long)(jc + lr) * e) + c)
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < kPieces; ++q) {
+      const int r = (tid + NTHR * q) >> 3;
+      xv[q] = (jc + r < nt && f0 < e) ? __ldg(reinterpret_cast<const float4*>(phk + (long long)(jc + r) * e + f0))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   };
-  load_chunk(0);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = static_cast<uint32_t>(misc[0]);
   const float inv_sqrt_e = rsqrtf((float)e);
   const uint64_t timeout_ns = args.timeout_ns;
   bool ok = true;
-  int phase = 0;
-  for (int jc = 0; jc < nt; jc += kTcCols) {
+  uint32_t tmem = 0;
+  // Chunk c's scores from TMEM buffer c % kTcAcc into the shared block:
+  // warp w < 8 reads lanes 32 (w % 4) .. +31 (K tiles) and columns
+  // 16 (w / 4) .. +15 (Q rows) of the buffer.
+  auto read_chunk = [&](int c) {
+    if (warp >= 8 || 16 * (warp >> 2) >= nq) return;
+    ok = mbar_wait(smem_u32(&bars[3 + c % kTcAcc]), (c / kTcAcc) & 1, abort, timeout_ns) && ok;
+    tc_fence_after();
+    if (!ok) return;
+    float v[16];
+    tmem_ld16(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)((c % kTcAcc) * 32 + 16 * (warp >> 2)), v);
+    tmem_ld_wait();
+    const int j = c * kTcCols + (warp & 3) * 32 + lane;
+    if (j < nt && VEDA_IN_BOUNDS(j < ntpad)) {
 #pragma unroll
-    for (int q = 0; q < KP / 8; ++q) {
-      const int c = lc0 + q;
-      store_split4(ahi + (c >> 3) * C::kAPanel, alo + (c >> 3) * C::kAPanel, lr, c & 7, xv[q]);
+      for (int r = 0; r < 16; ++r) {
+        const int q = 16 * (warp >> 2) + r;
+        if (q < nrows) s_scores[q * ntpad + j] = v[r] * inv_sqrt_e;
+      }
     }
+  };
+
+  load_stage(0);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  tmem = static_cast<uint32_t>(misc[0]);
+  for (int u = 0; u < nst; ++u) {
+    const int c = u / kP, p = u % kP;
+    if (p == 0 && c >= 2) read_chunk(c - 2);
+    // stage u % 3 is free once the products of stage u - 3 have completed
+    if (u >= kTcStages) ok = mbar_wait(smem_u32(&bars[u % kTcStages]), ((u - kTcStages) / kTcStages) & 1, abort,
+                                       timeout_ns) && ok;
+    uint8_t* ahi = smem + C::kOffA + (u % kTcStages) * C::kStage;
+    uint8_t* alo = ahi + C::kAPanel;
+#pragma unroll
+    for (int q = 0; q < kPieces; ++q) store_split4(ahi, alo, (tid + NTHR * q) >> 3, pc, xv[q]);
+    if (u + 1 < nst) load_stage(u + 1);   // overlaps the barrier and the products
     fence_proxy_async_smem();
     tc_fence_before();
     ok = __syncthreads_and(ok);
     if (!ok) break;
     if (tid == 0) {
       tc_fence_after();
-      constexpr uint32_t idesc = make_idesc_tf32(kTcCols, kTcRows);
+      const uint32_t idesc = make_idesc_tf32(kTcCols, nq);
       const uint64_t dah = make_sdesc_sw128(smem_u32(ahi), 16, 1024), dal = make_sdesc_sw128(smem_u32(alo), 16, 1024);
-      const uint64_t dbh = make_sdesc_sw128(smem_u32(bhi), 16, 1024), dbl = make_sdesc_sw128(smem_u32(blo), 16, 1024);
+      const uint64_t dbh = make_sdesc_sw128(smem_u32(bhi + p * C::kBPanel), 16, 1024);
+      const uint64_t dbl = make_sdesc_sw128(smem_u32(blo + p * C::kBPanel), 16, 1024);
+      const uint32_t acc = tmem + (uint32_t)((c % kTcAcc) * 32);
 #pragma unroll
-      for (int p = 0; p < KP / 32; ++p) {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t oa = (uint64_t)((p * C::kAPanel + kk * 32) >> 4);
-          const uint64_t ob = (uint64_t)((p * C::kBPanel + kk * 32) >> 4);
-          umma_tf32_ss(tmem, dah + oa, dbh + ob, idesc, (p > 0 || kk > 0) ? 1u : 0u);
-          umma_tf32_ss(tmem, dah + oa, dbl + ob, idesc, 1u);
-          umma_tf32_ss(tmem, dal + oa, dbh + ob, idesc, 1u);
-        }
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t off = (uint64_t)((kk * 32) >> 4);
+        umma_tf32_ss(acc, dah + off, dbh + off, idesc, (p > 0 || kk > 0) ? 1u : 0u);
+        umma_tf32_ss(acc, dah + off, dbl + off, idesc, 1u);
+        umma_tf32_ss(acc, dal + off, dbh + off, idesc, 1u);
       }
-      umma_commit(smem_u32(&bars[0]));
+      umma_commit(smem_u32(&bars[u % kTcStages]));
+      if (p == kP - 1) umma_commit(smem_u32(&bars[3 + c % kTcAcc]));
     }
-    if (jc + kTcCols < nt) load_chunk(jc + kTcCols);   // overlaps the products
-    ok = mbar_wait(smem_u32(&bars[0]), phase & 1, abort, timeout_ns) && ok;
-    ++phase;
-    tc_fence_after();
-    if (ok && warp < 4) {
-      float v[16];
-      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), v);
-      tmem_ld_wait();
-      const int j = jc + warp * 32 + lane;
-      if (j < nt && VEDA_IN_BOUNDS(j < ntpad)) {
-#pragma unroll
-        for (int r = 0; r < kTcRows; ++r)
-          if (r < nrows) s_scores[r * ntpad + j] = v[r] * inv_sqrt_e;
-      }
-    }
-    tc_fence_before();
-    ok = __syncthreads_and(ok);   // the A panels and TMEM are free for the next chunk
-    if (!ok) break;
   }
+  if (ok)
+    for (int c = max(0, nch - 2); c < nch; ++c) read_chunk(c);
   // Every MMA issued above completes before TMEM is released.
   if (tid == 0) {
-    umma_commit(smem_u32(&bars[1]));
+    umma_commit(smem_u32(&bars[7]));
     int dummy = 0;
-    mbar_wait(smem_u32(&bars[1]), 0, &dummy, timeout_ns);
+    mbar_wait(smem_u32(&bars[7]), 0, &dummy, timeout_ns);
   }
   tc_fence_before();
   ok = __syncthreads_and(ok);
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 32);
+    tmem_dealloc(tmem, kTcAcc * 32);
   }
   if (!ok) return;   // a wait ran out: the device error word reports it
-  select_rows<KPL>(G, args, s_scores, s_hist, qb, ntpad, nrows, nt, k, i0, idx_base, probs_base, warp, lane);
+  select_rows<KPL, NTHR / 32>(G, args, s_scores, s_hist, qb, ntpad, nrows, nt, k, i0, idx_base, probs_base, warp,
+                              lane);
 }
 
-// Which scoring kernel runs.  The tensor-core one for rows longer than 1,024
-// tiles (e <= 64): there the score product dominates and it is about 11%
-// faster end to end (245,760 tokens: 1.47 against 1.65 ms for estimator plus
-// selection).  Shorter rows keep the fp32 SIMT kernel, which needs fewer
-// registers and fits two CTAs per SM (Wan2.1-14B: 0.46 against 0.53 ms).
-static bool score_on_tensor_cores(int ntmax, int e) { return e <= 64 && ntmax > 1024; }
+// Which scoring kernel runs: the tensor-core one for feature widths up to 64
+// (every row length), the fp32 SIMT one for e = 128.
+static bool score_on_tensor_cores(int e) { return e <= 64; }
+
+// Threads of the tensor-core kernel: 16 warps for rows of up to 1,024 tiles
+// (at most 32 keys per lane in registers), 8 for longer rows.
+static int score_tc_threads(int ntmax) { return ntmax <= 1024 ? 512 : 256; }
 
 cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const float* desc_k,
                               const EstimatorWeights& wq, const EstimatorWeights& wk, int hidden,
@@ -487,24 +566,36 @@ cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const floa
   size_t smem;
   score_topk_config(G.ntmax, e, &qb, &ntpad, &smem);
   dim3 g2((G.ntmax + qb - 1) / qb, G.B * G.heads);
-  // keys per lane of the register bisection: the row length it covers is 32 x KPL
-  auto go = [&](auto kernel) -> cudaError_t {
+  auto go = [&](auto kernel, int threads) -> cudaError_t {
     cudaError_t e2 = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e2 != cudaSuccess) return e2;
-    kernel<<<g2, kScoreThreads, smem, s>>>(G, phi, e, qb, ntpad, args);
+    kernel<<<g2, threads, smem, s>>>(G, phi, e, qb, ntpad, args);
     return cudaGetLastError();
   };
-  if (score_on_tensor_cores(G.ntmax, e)) {
+  // keys per lane of the register bisection: the row length it covers is 32 x KPL
+  if (score_on_tensor_cores(e)) {
+    const int n = G.ntmax;
     if (e <= 32) {
-      if (G.ntmax <= 32 * 64) return go(score_topk_tc_kernel<64, 32>);
-      return go(score_topk_tc_kernel<0, 32>);
+      if (n <= 32 * 8) return go(score_topk_tc_kernel<8, 32, 512>, 512);
+      if (n <= 32 * 16) return go(score_topk_tc_kernel<16, 32, 512>, 512);
+      if (n <= 32 * 24) return go(score_topk_tc_kernel<24, 32, 512>, 512);
+      if (n <= 32 * 32) return go(score_topk_tc_kernel<32, 32, 512>, 512);
+      if (n <= 32 * 64) return go(score_topk_tc_kernel<64, 32, 256>, 256);
+      return go(score_topk_tc_kernel<0, 32, 256>, 256);
     }
-    if (G.ntmax <= 32 * 64) return go(score_topk_tc_kernel<64, 64>);
-    return go(score_topk_tc_kernel<0, 64>);
+    if (n <= 32 * 8) return go(score_topk_tc_kernel<8, 64, 512>, 512);
+    if (n <= 32 * 16) return go(score_topk_tc_kernel<16, 64, 512>, 512);
+    if (n <= 32 * 24) return go(score_topk_tc_kernel<24, 64, 512>, 512);
+    if (n <= 32 * 32) return go(score_topk_tc_kernel<32, 64, 512>, 512);
+    if (n <= 32 * 64) return go(score_topk_tc_kernel<64, 64, 256>, 256);
+    return go(score_topk_tc_kernel<0, 64, 256>, 256);
   }
-  if (G.ntmax <= 32 * 32) return go(score_topk_kernel<32>);
-  if (G.ntmax <= 32 * 64) return go(score_topk_kernel<64>);
-  return go(score_topk_kernel<0>);
+  if (G.ntmax <= 32 * 8) return go(score_topk_kernel<8>, kScoreThreads);
+  if (G.ntmax <= 32 * 16) return go(score_topk_kernel<16>, kScoreThreads);
+  if (G.ntmax <= 32 * 24) return go(score_topk_kernel<24>, kScoreThreads);
+  if (G.ntmax <= 32 * 32) return go(score_topk_kernel<32>, kScoreThreads);
+  if (G.ntmax <= 32 * 64) return go(score_topk_kernel<64>, kScoreThreads);
+  return go(score_topk_kernel<0>, kScoreThreads);
 }
 
 // Rows per CTA so that the score block fits beside the staging buffers in
@@ -512,11 +603,15 @@ cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const floa
 void score_topk_config(int ntmax, int e, int* qb, int* ntpad, size_t* smem) {
   const int pad = (ntmax + 3) & ~3;
   const bool radix = ntmax > 32 * 64;
+  const bool tc = score_on_tensor_cores(e);
+  const int nthr = score_tc_threads(ntmax);
+  auto tc_bytes = [&](int rows) {
+    return e <= 32 ? ScoreTcCfg<32>::smem_bytes(rows, pad, radix, nthr) : ScoreTcCfg<64>::smem_bytes(rows, pad, radix, nthr);
+  };
   int rows;
-  if (score_on_tensor_cores(ntmax, e)) {
-    const size_t fixed = e <= 32 ? ScoreTcCfg<32>::smem_bytes(0, pad, radix) : ScoreTcCfg<64>::smem_bytes(0, pad, radix);
-    rows = (int)(((size_t)227 * 1024 - fixed) / (4 * (size_t)pad));
-    if (rows > kTcRows) rows = kTcRows;
+  if (tc) {
+    rows = (int)(((size_t)227 * 1024 - tc_bytes(0)) / (4 * (size_t)pad));
+    if (rows > kTcMaxRows) rows = kTcMaxRows;
   } else {
     rows = (int)((140 * 1024) / (4 * (size_t)pad));
     if (rows > kQRows) rows = kQRows;
@@ -524,8 +619,8 @@ void score_topk_config(int ntmax, int e, int* qb, int* ntpad, size_t* smem) {
   if (rows < 1) rows = 1;
   *qb = rows;
   *ntpad = pad;
-  if (score_on_tensor_cores(ntmax, e))
-    *smem = e <= 32 ? ScoreTcCfg<32>::smem_bytes(rows, pad, radix) : ScoreTcCfg<64>::smem_bytes(rows, pad, radix);
+  if (tc)
+    *smem = tc_bytes(rows);
   else
     *smem = sizeof(float) * ((size_t)rows * pad + (size_t)e * kQRows + (size_t)e * kKChunk) +
             sizeof(uint32_t) * 8 * 256;
