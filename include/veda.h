@@ -154,7 +154,10 @@ veda_status veda_tripool_grid(const veda_problem* p, const void* x, float* desc,
 
 /* ---------------------------------------------------------------- steps 3-4: estimator + top-k */
 
-/* Bytes of workspace veda_tile_score_topk needs for estimator width e. */
+/* Bytes of workspace veda_tile_score_topk needs for estimator width e: the
+ * estimator features (2*B*heads*NT_max*e fp32) and, for e <= 64, the fp32
+ * score matrix [B, heads, NT_max, NT_max rounded up to a multiple of 4]
+ * (83 MB at the Wan2.1-14B 720p shape), each rounded up to 256 bytes. */
 veda_status veda_score_topk_workspace(const veda_problem* p, int32_t e, size_t* bytes);
 
 /* Distilled tile scoring and selection (section 2.1 "distilled tile scoring",

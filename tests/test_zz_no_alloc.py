@@ -6,8 +6,11 @@ loop that must not call cudaMalloc).
 The call goes straight through the C ABI (ctypes) and its results are
 compared with the workspace-taking veda_tile_score_topk on the same inputs,
 twice in a row on problems of different sizes, so the second call runs over
-whatever the first one left in the library's built-in scratch array.  The
-file is named to be collected last.
+whatever the first one left in the library's built-in scratch array.  On
+rows of more than 512 tiles the two entry points take different kernels (the
+fused one without a workspace, the score-matrix one with it), and the
+comparison checks that they select the same tiles.  The file is named to be
+collected last.
 """
 import ctypes
 
@@ -79,6 +82,34 @@ def test_noalloc_matches_workspace_entry_point_twice(V):
         # probabilities agree within the tolerance the parity tests use.
         assert torch.equal(idx, ref_idx)
         np.testing.assert_allclose(probs.cpu().numpy(), ref_probs.cpu().numpy(), rtol=PROBS_REL, atol=PROBS_ABS)
+
+
+# Rows of more than 512 tiles: the workspace entry point scores through the
+# fp32 score matrix it keeps in the workspace (tensor-core GEMM, then one warp
+# per row), the no-alloc one through the fused kernel that keeps each CTA's
+# scores in shared memory.  Both form the same tf32 products in the same order
+# and select from the same fp32 scores, so the selections are identical.
+LONG_ROWS = [
+    Workload(name="rows720", T=24, H=40, W=44, B=1, heads=2, d=64, S=64, tilings=((4, 4, 4), (2, 4, 8)),
+             keep=0.05, hidden=128, e=32, bias="rff"),
+    Workload(name="rows770", T=26, H=42, W=40, B=1, heads=2, d=128, S=64, tilings=((4, 4, 4), (2, 4, 8)),
+             keep=0.05, hidden=256, e=64, bias="rff"),
+    Workload(name="rows1760", T=39, H=41, W=58, B=1, heads=2, d=64, S=64, tilings=((4, 4, 4), (2, 4, 8)),
+             keep=0.05, hidden=128, e=32, bias="rff"),
+    Workload(name="rows2200", T=50, H=44, W=60, B=1, heads=2, d=64, S=64, tilings=((4, 4, 4), (2, 4, 8)),
+             keep=0.05, hidden=128, e=32, bias="rff"),
+]
+
+
+@pytest.mark.parametrize("w", LONG_ROWS, ids=[w.name for w in LONG_ROWS])
+def test_noalloc_fused_kernel_matches_score_matrix_path(V, w):
+    p, dq, dk, mlp, _wts, k_max = _case(V, w, 5)
+    assert p.nt_max > 512
+    ref_idx, ref_probs = _reference(V, p, dq, dk, mlp, w.keep, k_max)
+    idx, probs = _noalloc_c_call(V, p, dq, dk, mlp, w.keep, k_max)
+    V.veda_sync_status()
+    assert torch.equal(idx, ref_idx)
+    np.testing.assert_allclose(probs.cpu().numpy(), ref_probs.cpu().numpy(), rtol=PROBS_REL, atol=PROBS_ABS)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(V):

@@ -99,9 +99,13 @@ cudaError_t launch_estimator(const Geometry& G, const float* dq, const float* dk
                              const EstimatorWeights& wk, int hidden, int e, float* phi, float* hid,
                              uint64_t timeout_ns, cudaStream_t s);
 void score_topk_config(int ntmax, int e, int* qb, int* ntpad, size_t* smem);
+// Scoring and selection.  phi: the estimator features, 2*B*heads*NT_max*e
+// floats.  scores: room for the fp32 score matrix (score_matrix_bytes), or
+// NULL, in which case each CTA keeps its block of scores in shared memory.
+size_t score_matrix_bytes(const Geometry& G, int e);
 cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const float* desc_k,
                               const EstimatorWeights& wq, const EstimatorWeights& wk, int hidden,
-                              int e, float* phi, const TopkArgs& args, cudaStream_t s);
+                              int e, float* phi, float* scores, const TopkArgs& args, cudaStream_t s);
 
 size_t sparse_attn_smem_bytes(int d, int S, int k_max);
 void sparse_attn_config(int d, int S, int k_max, int* k_stages, int* v_stages, size_t* smem);

@@ -3,21 +3,27 @@
 // tile scores form a row-wise distribution over K tiles; section 4 / news
 // page: keep the top ~5-10% of tiles).
 //
-// Two launches:
+// The estimator, then one of two selection paths:
 //   estimator_kernel  phi = W2 relu(W1 desc + b1) + b2 for every Q and K tile,
 //                     on the tensor cores at fp32 accuracy (estimator.cu),
 //                     written to the workspace;
-//   score_topk_tc_kernel (scores on the tensor cores; feature widths e up
-//                     to 64) or score_topk_kernel (fp32 SIMT scores, e = 128)
-//                     per block of Q-tile rows: s = phi_q phi_k^T / sqrt(e)
-//                     into shared memory, optional row softmax, then the
-//                     exact k-th largest score per row and an ascending
-//                     compaction of the winners.  Rows of up to 2048 tiles
-//                     find the k-th largest by bisection over order-preserving
-//                     32-bit keys held in registers (one warp per row, a
-//                     compare-and-count per step, no shared-memory traffic);
-//                     longer rows use a 4-pass radix select over shared
-//                     histograms.
+//   rows of more than 512 tiles, e <= 64, with the score matrix in the
+//   workspace:
+//     score_gemm_kernel  s = phi_q phi_k^T / sqrt(e) for a head's whole
+//                        [NT, NT] block, on the tensor cores, into the
+//                        workspace;
+//     topk_rows_kernel   one warp per row: optional row softmax, the exact
+//                        k-th largest score and an ascending compaction of
+//                        the winners;
+//   otherwise (shorter rows, e = 128, or no room for the matrix):
+//     score_topk_tc_kernel (scores on the tensor cores; e up to 64) or
+//                        score_topk_kernel (fp32 SIMT scores, e = 128) per
+//                        block of Q-tile rows, the scores kept in shared
+//                        memory, then the same select.
+// Rows of up to 2048 tiles find the k-th largest by bisection over
+// order-preserving 32-bit keys held in registers (one warp per row, a
+// compare-and-count per step); longer rows use a 4-pass radix select over
+// shared histograms.
 // Scores stay fp32 end to end so that selections only differ from an exact
 // evaluation on genuine near-ties.
 #include "veda_common.cuh"
@@ -548,6 +554,225 @@ __global__ void __launch_bounds__(NTHR, 1)
                               lane);
 }
 
+// ---------------------------------------------------------------------------
+// Score matrix on the tensor cores, for callers whose workspace holds it:
+// S[b, h, i, j] = <phi_q[i], phi_k[j]> / sqrt(e) for i, j < NT_h, fp32
+// [B*heads][NT_max][ntpad].  A CTA takes 128 Q rows of one head (the MMA's N)
+// and walks the head's K tiles in chunks of 128 (the MMA's M) with the same
+// tcgen05 kind::tf32 split and the same product order as the kernel above
+// (S^T = phi_k phi_q^T, hi*hi, hi*lo, lo*hi per 8-feature step), so the two
+// give the same scores.  The next chunk's phi_k rows are loaded into
+// registers (a warp reads two whole rows per load) while the current chunk is
+// multiplied; two A stages and two TMEM accumulators let chunk c's products
+// run while chunk c - 1 is read back and stored.  Warp w reads K tiles
+// 32 (w % 4) .. +31 and Q rows 64 (w / 4) .. +63 of the accumulator and
+// stores 32 consecutive scores of one row per instruction.
+// ---------------------------------------------------------------------------
+constexpr int kSgRows = 128;      // Q rows per CTA: the MMA's N
+constexpr int kSgThreads = 256;
+
+template <int KP>
+struct ScoreGemmCfg {
+  static constexpr int kPanels = KP / 32;
+  static constexpr int kAPanel = kTcCols * 128;          // 128 K-tile rows x 32 fp32
+  static constexpr int kBPanel = kSgRows * 128;          // 128 Q rows x 32 fp32
+  static constexpr int kStage = 2 * kPanels * kAPanel;   // hi panels, then lo panels, of one chunk
+  static constexpr int kOffA = 0;                        // two stages
+  static constexpr int kOffBhi = 2 * kStage;
+  static constexpr int kOffBlo = kOffBhi + kPanels * kBPanel;
+  static constexpr int kOffBar = kOffBlo + kPanels * kBPanel;   // A stage free [2], accumulator full [2], drain; misc
+  static constexpr size_t kSmem = 1024 + kOffBar + 64;
+};
+
+template <int KP>
+__global__ void __launch_bounds__(kSgThreads, 1)
+    score_gemm_kernel(const __grid_constant__ Geometry G, const float* __restrict__ phi, int e, int ntpad,
+                      float* __restrict__ S, uint64_t timeout_ns) {
+  using C = ScoreGemmCfg<KP>;
+  constexpr int kP = C::kPanels;
+  constexpr int kRowPieces = KP / 4;                             // 16-byte pieces of a phi row
+  constexpr int kPieces = kTcCols * kRowPieces / kSgThreads;     // of a chunk, per thread
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int bh = blockIdx.y;
+  const int nt = G.g[bh % G.heads].nt;
+  const int i0 = blockIdx.x * kSgRows;
+  if (i0 >= nt) return;   // CTA-uniform, before any barrier or TMEM use
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nrows = min(kSgRows, nt - i0);
+  uint8_t* bhi = smem + C::kOffBhi;
+  uint8_t* blo = smem + C::kOffBlo;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);   // [0,2) A free, [2,4) acc full, [4] drain
+  int* misc = reinterpret_cast<int*>(bars + 5);                        // [0] TMEM base, [1] abort
+  volatile int* abort = misc + 1;
+  const float* phq = phi + ((long long)bh * G.ntmax + i0) * e;
+  const float* phk = phi + (((long long)G.B * G.heads + bh) * G.ntmax) * e;
+  if (tid == 0) {
+    for (int b = 0; b < 5; ++b) mbar_init(smem_u32(&bars[b]), 1);
+    misc[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&misc[0]), 256);
+    tmem_relinquish();
+  }
+  // B: the block's phi_q rows, split (rows past nrows and features past e are zero)
+  for (int t = tid; t < kSgRows * kRowPieces; t += kSgThreads) {
+    const int r = t / kRowPieces, c4 = t % kRowPieces;
+    const float4 v = (r < nrows && 4 * c4 < e) ? __ldg(reinterpret_cast<const float4*>(phq + (long long)r * e) + c4)
+                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+    store_split4(bhi + (c4 >> 3) * C::kBPanel, blo + (c4 >> 3) * C::kBPanel, r, c4 & 7, v);
+  }
+  // A: piece tid + 256 q of a chunk is K-tile row (tid + 256 q) / (KP / 4),
+  // 16-byte piece (tid % (KP / 4)) of that row.
+  float4 xv[kPieces];
+  auto load_chunk = [&](int jc) {
+#pragma unroll
+    for (int q = 0; q < kPieces; ++q) {
+      const int t = tid + kSgThreads * q, r = t / kRowPieces, c4 = t % kRowPieces;
+      xv[q] = (jc + r < nt && 4 * c4 < e) ? __ldg(reinterpret_cast<const float4*>(phk + (long long)(jc + r) * e) + c4)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  const int nch = (nt + kTcCols - 1) / kTcCols;
+  load_chunk(0);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+  const float inv_sqrt_e = rsqrtf((float)e);
+  bool ok = true;
+  auto store_chunk = [&](int c) {
+    ok = mbar_wait(smem_u32(&bars[2 + (c & 1)]), (c >> 1) & 1, abort, timeout_ns) && ok;
+    tc_fence_after();
+    if (!ok) return;
+    const int j = c * kTcCols + (warp & 3) * 32 + lane;
+    float* row0 = S + ((long long)bh * G.ntmax + i0) * ntpad + j;
+#pragma unroll
+    for (int cb = 0; cb < 2; ++cb) {
+      const int q0 = (warp >> 2) * 64 + cb * 32;
+      float v[32];
+      tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)((c & 1) * kSgRows + q0), v);
+      tmem_ld_wait();
+      if (j < nt && VEDA_IN_BOUNDS(j < ntpad)) {
+#pragma unroll
+        for (int r = 0; r < 32; ++r)
+          if (q0 + r < nrows) row0[(long long)(q0 + r) * ntpad] = v[r] * inv_sqrt_e;
+      }
+    }
+  };
+  for (int c = 0; c < nch; ++c) {
+    const int st = c & 1;
+    // A stage st is free once the products of chunk c - 2 have completed
+    if (c >= 2) ok = mbar_wait(smem_u32(&bars[st]), ((c - 2) >> 1) & 1, abort, timeout_ns) && ok;
+    uint8_t* ahi = smem + C::kOffA + st * C::kStage;
+    uint8_t* alo = ahi + kP * C::kAPanel;
+#pragma unroll
+    for (int q = 0; q < kPieces; ++q) {
+      const int t = tid + kSgThreads * q, r = t / kRowPieces, c4 = t % kRowPieces;
+      store_split4(ahi + (c4 >> 3) * C::kAPanel, alo + (c4 >> 3) * C::kAPanel, r, c4 & 7, xv[q]);
+    }
+    if (c + 1 < nch) load_chunk((c + 1) * kTcCols);   // overlaps the products
+    fence_proxy_async_smem();
+    tc_fence_before();
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t idesc = make_idesc_tf32(kTcCols, kSgRows);
+      const uint32_t acc = tmem + (uint32_t)(st * kSgRows);
+#pragma unroll
+      for (int p = 0; p < kP; ++p) {
+        const uint64_t dah = make_sdesc_sw128(smem_u32(ahi + p * C::kAPanel), 16, 1024);
+        const uint64_t dal = make_sdesc_sw128(smem_u32(alo + p * C::kAPanel), 16, 1024);
+        const uint64_t dbh = make_sdesc_sw128(smem_u32(bhi + p * C::kBPanel), 16, 1024);
+        const uint64_t dbl = make_sdesc_sw128(smem_u32(blo + p * C::kBPanel), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t off = (uint64_t)((kk * 32) >> 4);
+          umma_tf32_ss(acc, dah + off, dbh + off, idesc, (p > 0 || kk > 0) ? 1u : 0u);
+          umma_tf32_ss(acc, dah + off, dbl + off, idesc, 1u);
+          umma_tf32_ss(acc, dal + off, dbh + off, idesc, 1u);
+        }
+      }
+      umma_commit(smem_u32(&bars[st]));
+      umma_commit(smem_u32(&bars[2 + st]));
+    }
+    if (c >= 1) store_chunk(c - 1);   // runs while chunk c is multiplied
+  }
+  if (ok) store_chunk(nch - 1);
+  // Every MMA issued above completes before TMEM is released.
+  if (tid == 0) {
+    umma_commit(smem_u32(&bars[4]));
+    int dummy = 0;
+    mbar_wait(smem_u32(&bars[4]), 0, &dummy, timeout_ns);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// Row softmax and top-k from the score matrix in the workspace: one warp per
+// Q-tile row, eight rows per CTA; the select is the one above, reading the
+// row's scores from global memory (a warp loads 32 consecutive scores).
+constexpr int kTrWarps = 8;
+
+template <int KPL>
+__global__ void __launch_bounds__(kTrWarps * 32)
+    topk_rows_kernel(const __grid_constant__ Geometry G, const float* __restrict__ S, int ntpad,
+                     const __grid_constant__ TopkArgs args) {
+  extern __shared__ uint32_t s_hist_rows[];   // radix select only: [8][256]
+  const int bh = blockIdx.y;
+  const int h = bh % G.heads;
+  const int nt = G.g[h].nt;
+  const int i0 = blockIdx.x * kTrWarps;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t* idx_base = args.idx + ((long long)bh * G.ntmax) * args.k_max;
+  float* probs_base = args.probs ? args.probs + ((long long)bh * G.ntmax) * G.ntmax : nullptr;
+  const int nrows = max(0, min(kTrWarps, nt - i0));
+  select_rows<KPL, kTrWarps>(G, args, S + ((long long)bh * G.ntmax + i0) * ntpad, s_hist_rows, kTrWarps, ntpad, nrows,
+                             nt, args.k_per_head[h], i0, idx_base, probs_base, warp, lane);
+}
+
+// Bytes of the score matrix in the workspace, 0 when the fused kernels score:
+// for e = 128, and for rows of up to 512 tiles, where the fused kernel is
+// faster (Wan2.1-1.3B: 0.062 against 0.073 ms for estimator plus selection;
+// Wan2.1-14B, 720 tiles: 0.314 against 0.265 ms).
+size_t score_matrix_bytes(const Geometry& G, int e) {
+  if (e > 64 || G.ntmax <= 512) return 0;
+  return sizeof(float) * (size_t)G.B * G.heads * G.ntmax * (size_t)((G.ntmax + 3) & ~3);
+}
+
+static cudaError_t launch_score_matrix_topk(const Geometry& G, int e, const float* phi, float* S,
+                                            const TopkArgs& args, cudaStream_t s) {
+  const int ntpad = (G.ntmax + 3) & ~3;
+  const dim3 g1((G.ntmax + kSgRows - 1) / kSgRows, G.B * G.heads);
+  auto gemm = [&](auto kernel, size_t smem) -> cudaError_t {
+    cudaError_t e2 = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e2 != cudaSuccess) return e2;
+    kernel<<<g1, kSgThreads, smem, s>>>(G, phi, e, ntpad, S, args.timeout_ns);
+    return cudaGetLastError();
+  };
+  cudaError_t err = e <= 32 ? gemm(score_gemm_kernel<32>, ScoreGemmCfg<32>::kSmem)
+                            : gemm(score_gemm_kernel<64>, ScoreGemmCfg<64>::kSmem);
+  if (err != cudaSuccess) return err;
+  const dim3 g2((G.ntmax + kTrWarps - 1) / kTrWarps, G.B * G.heads);
+  const int n = G.ntmax;
+  auto rows = [&](auto kernel, size_t smem) -> cudaError_t {
+    kernel<<<g2, kTrWarps * 32, smem, s>>>(G, S, ntpad, args);
+    return cudaGetLastError();
+  };
+  if (n <= 32 * 8) return rows(topk_rows_kernel<8>, 0);
+  if (n <= 32 * 16) return rows(topk_rows_kernel<16>, 0);
+  if (n <= 32 * 24) return rows(topk_rows_kernel<24>, 0);
+  if (n <= 32 * 32) return rows(topk_rows_kernel<32>, 0);
+  if (n <= 32 * 64) return rows(topk_rows_kernel<64>, 0);
+  return rows(topk_rows_kernel<0>, sizeof(uint32_t) * kTrWarps * 256);
+}
+
 // Which scoring kernel runs: the tensor-core one for feature widths up to 64
 // (every row length), the fp32 SIMT one for e = 128.
 static bool score_on_tensor_cores(int e) { return e <= 64; }
@@ -558,9 +783,10 @@ static int score_tc_threads(int ntmax) { return ntmax <= 1024 ? 512 : 256; }
 
 cudaError_t launch_score_topk(const Geometry& G, const float* desc_q, const float* desc_k,
                               const EstimatorWeights& wq, const EstimatorWeights& wk, int hidden,
-                              int e, float* phi, const TopkArgs& args, cudaStream_t s) {
+                              int e, float* phi, float* scores, const TopkArgs& args, cudaStream_t s) {
   cudaError_t err = launch_estimator(G, desc_q, desc_k, wq, wk, hidden, e, phi, nullptr, args.timeout_ns, s);
   if (err != cudaSuccess) return err;
+  if (scores != nullptr && score_matrix_bytes(G, e) > 0) return launch_score_matrix_topk(G, e, phi, scores, args, s);
 
   int qb, ntpad;
   size_t smem;

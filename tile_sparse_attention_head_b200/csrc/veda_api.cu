@@ -164,9 +164,13 @@ veda_status encode_grid_tiles(const Geometry& G, const void* ptr, const HeadGeom
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
-size_t score_ws_bytes(const Geometry& G, int e) {
+// The estimator features: 2*B*heads*NT_max*e floats.
+size_t phi_ws_bytes(const Geometry& G, int e) {
   return round256(sizeof(float) * 2 * (size_t)G.B * G.heads * G.ntmax * e);
 }
+
+// veda_tile_score_topk's workspace: the features, then the score matrix.
+size_t score_ws_bytes(const Geometry& G, int e) { return phi_ws_bytes(G, e) + round256(score_matrix_bytes(G, e)); }
 
 size_t map_rowmax_bytes(const Geometry& G, int R) {
   return round256(sizeof(float) * (size_t)G.B * G.heads * R * G.ntmax * G.S);
@@ -329,8 +333,11 @@ veda_status veda_tile_score_topk(const veda_problem* p, const float* desc_q, con
   args.timeout_ns = g_timeout_ns;
   EstimatorWeights wq{mlp_q->w1, mlp_q->b1, mlp_q->w2, mlp_q->b2};
   EstimatorWeights wk{mlp_k->w1, mlp_k->b1, mlp_k->w2, mlp_k->b2};
-  cudaError_t ce = launch_score_topk(G, desc_q, desc_k, wq, wk, hidden, e, static_cast<float*>(workspace), args,
-                                     (cudaStream_t)stream);
+  float* phi = static_cast<float*>(workspace);
+  float* scores = score_matrix_bytes(G, e) > 0
+                      ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + phi_ws_bytes(G, e))
+                      : nullptr;
+  cudaError_t ce = launch_score_topk(G, desc_q, desc_k, wq, wk, hidden, e, phi, scores, args, (cudaStream_t)stream);
   if (ce != cudaSuccess) return cuda_fail(ce, "veda_tile_score_topk");
   return ok();
 }
@@ -425,7 +432,7 @@ veda_status veda_tile_score_topk_noalloc(const veda_problem* p, const float* des
   if (!aligned16(desc_q) || !aligned16(desc_k) || !aligned16(idx) || (probs && !aligned16(probs)))
     return fail(VEDA_ERR_INVALID_ARG, "tensor arguments must be 16-byte aligned");
   const int e = mlp_q->e, hidden = mlp_q->hidden;
-  const size_t need = score_ws_bytes(G, e);
+  const size_t need = phi_ws_bytes(G, e);
   if (need > kNoAllocScratchBytes)
     return fail(VEDA_ERR_UNSUPPORTED,
                 "estimator scratch of %zu bytes exceeds the built-in %zu bytes (2*B*heads*NT_max*e floats); "
@@ -449,7 +456,7 @@ veda_status veda_tile_score_topk_noalloc(const veda_problem* p, const float* des
   args.timeout_ns = g_timeout_ns;
   EstimatorWeights wq{mlp_q->w1, mlp_q->b1, mlp_q->w2, mlp_q->b2};
   EstimatorWeights wk{mlp_k->w1, mlp_k->b1, mlp_k->w2, mlp_k->b2};
-  cudaError_t ce = launch_score_topk(G, desc_q, desc_k, wq, wk, hidden, e, scratch, args, (cudaStream_t)stream);
+  cudaError_t ce = launch_score_topk(G, desc_q, desc_k, wq, wk, hidden, e, scratch, nullptr, args, (cudaStream_t)stream);
   if (ce != cudaSuccess) return cuda_fail(ce, "veda_tile_score_topk_noalloc");
   return ok();
 }
