@@ -42,11 +42,18 @@ __device__ __forceinline__ uint32_t float_key(float f) {
 
 // k-th largest key of a row by bisection: each lane holds keys of columns
 // lane, lane + 32, ... (KPL of them, 0 past the row end; every real key is
-// above 0).  Returns the key value t and, in *gt, the number of keys above t.
-// Invariant: count(key >= lo) >= k > count(key >= hi); a midpoint with exactly
-// k keys at or above it ends the search early.
+// above 0).  Invariant: count(key >= lo) = c_lo >= k > count(key >= hi) =
+// c_hi; a midpoint with exactly k keys at or above it ends the search early.
+// Returns the k-th largest key t.  *exact is set when exactly k keys are at
+// or above t (then those are the selection); otherwise *gt is the number of
+// keys above t, and the selection takes the first k - *gt keys equal to t.
+// With a candidate buffer (`cand`, 64 entries owned by the warp), once at
+// most 64 keys lie in [lo, hi) they are gathered there and the search goes on
+// over those two per lane instead of all KPL keys per lane; the result is
+// the same.
 template <int KPL>
-__device__ __forceinline__ uint32_t kth_key_bisect(const uint32_t (&key)[KPL], int nt, int k, int lane, int* gt) {
+__device__ __forceinline__ uint32_t kth_key_bisect(const uint32_t (&key)[KPL], int nt, int k, int lane, int* gt,
+                                                   bool* exact, uint32_t* cand) {
   uint32_t kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
   for (int i = 0; i < KPL; ++i)
@@ -56,36 +63,71 @@ __device__ __forceinline__ uint32_t kth_key_bisect(const uint32_t (&key)[KPL], i
     }
   kmin = __reduce_min_sync(0xffffffffu, kmin);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
-  auto count_ge = [&](uint32_t t) {
+  uint64_t lo = kmin, hi = (uint64_t)kmax + 1;
+  int c_lo = nt, c_hi = 0;
+  *exact = false;
+  // Phase 1: all keys.
+  while (hi - lo > 1 && (cand == nullptr || c_lo - c_hi > 64)) {
+    const uint32_t mid = (uint32_t)(lo + ((hi - lo) >> 1));
     int c = 0;
 #pragma unroll
-    for (int i = 0; i < KPL; ++i) c += key[i] >= t ? 1 : 0;
-    return (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
-  };
-  uint64_t lo = kmin, hi = (uint64_t)kmax + 1;
-  uint32_t t = 0;
-  bool found = false;
-  while (hi - lo > 1) {
-    const uint64_t mid = lo + ((hi - lo) >> 1);
-    const int c = count_ge((uint32_t)mid);
+    for (int i = 0; i < KPL; ++i) c += key[i] >= mid ? 1 : 0;
+    c = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
     if (c == k) {   // exactly the k largest are >= mid: t is the smallest of them
       uint32_t m = 0xffffffffu;
 #pragma unroll
       for (int i = 0; i < KPL; ++i)
-        if (key[i] >= (uint32_t)mid) m = min(m, key[i]);
-      t = __reduce_min_sync(0xffffffffu, m);
-      found = true;
-      break;
+        if (key[i] >= mid) m = min(m, key[i]);
+      *exact = true;
+      return __reduce_min_sync(0xffffffffu, m);
     }
-    if (c > k) lo = mid;
-    else hi = mid;
+    if (c > k) {
+      lo = mid;
+      c_lo = c;
+    } else {
+      hi = mid;
+      c_hi = c;
+    }
   }
-  if (!found) t = (uint32_t)lo;
-  int c = 0;
+  if (hi - lo > 1) {
+    // Phase 2: the c_lo - c_hi <= 64 keys in [lo, hi), gathered in order of
+    // appearance; every key outside is either counted in c_hi or below lo.
+    int base = 0;
 #pragma unroll
-  for (int i = 0; i < KPL; ++i) c += key[i] > t ? 1 : 0;
-  *gt = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
-  return t;
+    for (int i = 0; i < KPL; ++i) {
+      if (i * 32 >= nt) break;   // warp-uniform
+      const bool in = i * 32 + lane < nt && key[i] >= lo && key[i] < hi;
+      const unsigned m = __ballot_sync(0xffffffffu, in);
+      if (in) cand[base + __popc(m & ((1u << lane) - 1u))] = key[i];
+      base += __popc(m);
+    }
+    __syncwarp();
+    const uint32_t k0 = lane < base ? cand[lane] : 0u, k1 = lane + 32 < base ? cand[lane + 32] : 0u;
+    __syncwarp();   // the buffer is free for the warp's next row
+    const int above = c_hi;   // keys at or above the bracket, none of them gathered
+    while (hi - lo > 1) {
+      const uint32_t mid = (uint32_t)(lo + ((hi - lo) >> 1));
+      const int c = above + (int)__reduce_add_sync(0xffffffffu, (unsigned)((k0 >= mid) + (k1 >= mid)));
+      if (c == k) {
+        uint32_t m = 0xffffffffu;
+        if (k0 >= mid) m = k0;
+        if (k1 >= mid) m = min(m, k1);
+        *exact = true;
+        return __reduce_min_sync(0xffffffffu, m);
+      }
+      if (c > k) {
+        lo = mid;
+        c_lo = c;
+      } else {
+        hi = mid;
+        c_hi = c;
+      }
+    }
+  }
+  // hi = lo + 1: t = lo, count(key >= t) = c_lo, count(key > t) = c_hi.
+  *exact = c_lo == k;
+  *gt = c_hi;
+  return (uint32_t)lo;
 }
 
 constexpr int kScoreThreads = 256;
@@ -98,7 +140,8 @@ constexpr int kQRows = 16;         // most Q-tile rows per CTA (the score tile i
 template <int KPL, int NWARPS>
 __device__ __forceinline__ void select_rows(const Geometry& G, const TopkArgs& args, const float* s_scores,
                                             uint32_t* s_hist, int qb, int ntpad, int nrows, int nt, int k, int i0,
-                                            int32_t* idx_base, float* probs_base, int warp, int lane) {
+                                            int32_t* idx_base, float* probs_base, int warp, int lane,
+                                            uint32_t* cand = nullptr) {
   uint32_t* hist = s_hist + warp * 256;
   for (int r = warp; r < qb; r += NWARPS) {
     const int i = i0 + r;
@@ -138,12 +181,28 @@ __device__ __forceinline__ void select_rows(const Geometry& G, const TopkArgs& a
         key[i] = c < nt ? float_key(srow[c]) : 0u;
       }
       int gt = 0;
-      prefix = kth_key_bisect(key, nt, k, lane, &gt);
+      bool exact = false;
+      prefix = kth_key_bisect(key, nt, k, lane, &gt, &exact, cand);
       remaining = k - gt;
-      // Every key above the k-th largest and the first `remaining` keys equal
-      // to it (smallest tile indices), in ascending column order; column
-      // i * 32 + lane is key[i] of this lane.
       int out = 0, eq_taken = 0;
+      if (exact) {
+        // Exactly k keys are >= the k-th largest: take them all, in ascending
+        // column order (column i * 32 + lane is key[i] of this lane).
+#pragma unroll
+        for (int i = 0; i < (KPL > 0 ? KPL : 1); ++i) {
+          if (i * 32 >= nt) break;   // warp-uniform
+          const int c = i * 32 + lane;
+          const bool take = c < nt && key[i] >= prefix;
+          const unsigned tmask = __ballot_sync(0xffffffffu, take);
+          const int pos = out + __popc(tmask & ((1u << lane) - 1u));
+          if (take && pos < k && VEDA_IN_BOUNDS(c < nt && pos < args.k_max)) irow[pos] = c;
+          out += __popc(tmask);
+        }
+        for (int c = k + lane; c < args.k_max; c += 32) irow[c] = -1;
+        continue;
+      }
+      // Every key above the k-th largest and the first `remaining` keys equal
+      // to it (smallest tile indices), in ascending column order.
 #pragma unroll
       for (int i = 0; i < (KPL > 0 ? KPL : 1); ++i) {
         if (i * 32 >= nt) break;   // warp-uniform
@@ -725,6 +784,7 @@ __global__ void __launch_bounds__(kTrWarps * 32)
     topk_rows_kernel(const __grid_constant__ Geometry G, const float* __restrict__ S, int ntpad,
                      const __grid_constant__ TopkArgs args) {
   extern __shared__ uint32_t s_hist_rows[];   // radix select only: [8][256]
+  __shared__ uint32_t s_cand[kTrWarps][64];   // the bisection's candidate buffers
   const int bh = blockIdx.y;
   const int h = bh % G.heads;
   const int nt = G.g[h].nt;
@@ -734,7 +794,7 @@ __global__ void __launch_bounds__(kTrWarps * 32)
   float* probs_base = args.probs ? args.probs + ((long long)bh * G.ntmax) * G.ntmax : nullptr;
   const int nrows = max(0, min(kTrWarps, nt - i0));
   select_rows<KPL, kTrWarps>(G, args, S + ((long long)bh * G.ntmax + i0) * ntpad, s_hist_rows, kTrWarps, ntpad, nrows,
-                             nt, args.k_per_head[h], i0, idx_base, probs_base, warp, lane);
+                             nt, args.k_per_head[h], i0, idx_base, probs_base, warp, lane, s_cand[warp]);
 }
 
 // Bytes of the score matrix in the workspace, 0 when the fused kernels score:
