@@ -3,6 +3,8 @@
 The launch picks kernel variants from the problem size, and the benchmark
 workloads reach variants that the small parity cases do not:
 
+* rows of more than 512 tiles score through the fp32 score matrix in the
+  workspace (tensor-core GEMM, then one warp per row), including B = 2;
 * top-k over rows of 257-512, 513-768 and 769-1,024 tiles: the register
   bisection with 16, 24 and 32 keys per lane (the Wan2.1-1.3B shape has up to
   336 tiles per head, the Wan2.1-14B shape 720), with every feature width the
@@ -97,6 +99,8 @@ TOPK_CASES = [
     wl("topk600e128", (24, 40, 40), 1, 1, 64, 64, [(4, 4, 4)], 0.05, 128, 128, "rff"),
     # 770 and 715 tiles at d = 128: 32 keys per lane, e = 64
     wl("topk770", (26, 42, 40), 1, 2, 128, 64, [(4, 4, 4), (2, 4, 8)], 0.05, 256, 64, "rff"),
+    # B = 2 with rows of 660 and 720 tiles: the score-matrix path's batch and head offsets
+    wl("topk720b2", (24, 40, 44), 2, 2, 64, 64, [(2, 4, 8), (4, 4, 4)], 0.05, 128, 32, "rff"),
     # 1,650 tiles: the 64-keys-per-lane register bisection
     wl("topk1650", (39, 41, 58), 1, 2, 64, 64, [(4, 4, 4), (2, 4, 8)], 0.05, 128, 32, "rff"),
     # 2,145 and 2,200 tiles: the radix select
