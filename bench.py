@@ -375,7 +375,15 @@ def attention_sustained(V, p, att, qd, kd, vd, out, args, flops, local):
     torch.cuda.synchronize()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1) / n
-    return {"launches": n, "ms_per_launch": ms, "tflops": flops / (ms * 1e-3) / 1e12, "clocks": clk}
+    # Operand bytes each launch streams from L2 into shared memory: every kept
+    # (Q tile, K tile) pair fetches its K and V tile, every Q tile is fetched
+    # once (the kept pairs follow from the kept-tile FLOPs, 4 S^2 d per pair).
+    tile_bytes = p.S * p.d * 2
+    pairs = flops / (4.0 * p.S * p.S * p.d)
+    q_tiles = p.B * sum(p.nt_per_head)
+    l2_bytes = pairs * 2 * tile_bytes + q_tiles * tile_bytes
+    return {"launches": n, "ms_per_launch": ms, "tflops": flops / (ms * 1e-3) / 1e12, "clocks": clk,
+            "l2_to_smem_bytes_per_launch": l2_bytes, "l2_to_smem_tb_per_s": l2_bytes / (ms * 1e-3) / 1e12}
 
 
 def backward_measure(V, w, p, att, qd, kd, vd, args, flops, rank, dev):
