@@ -386,6 +386,57 @@ def attention_sustained(V, p, att, qd, kd, vd, out, args, flops, local):
             "l2_to_smem_bytes_per_launch": l2_bytes, "l2_to_smem_tb_per_s": l2_bytes / (ms * 1e-3) / 1e12}
 
 
+def overlap_measure(V, w, qd, kd, vd, mlp, out_ref, args, dev):
+    """Prototype of selection overlapped with attention: the heads split into
+    args.overlap_groups groups (one Problem and VedaAttention each, on head
+    slices of the same tensors), groups alternating between two streams, so
+    that group g+1's TripPool, estimator and top-k can run beside group g's
+    attention.  Returns ms per layer (CUDA events around the whole layer,
+    after both streams join) and whether the output matches the one-stream
+    layer bit for bit."""
+    if args.layout != "grid" or w.B != 1:
+        return {"skipped": "grid layout with B = 1 only (head slices must be contiguous)"}
+    G = args.overlap_groups
+    bounds = [round(i * w.heads / G) for i in range(G + 1)]
+    groups = []
+    for g in range(G):
+        h0, h1 = bounds[g], bounds[g + 1]
+        pg = V.Problem(w.B, h1 - h0, w.d, w.S, (w.T, w.H, w.W), w.tilings[h0:h1])
+        mg = tuple(t[h0:h1].contiguous() for t in mlp)
+        att = V.VedaAttention(pg, mg, mg, w.keep, device=dev, layout="grid")
+        sl = lambda t: t[:, h0:h1]
+        groups.append((pg, att, sl(qd), sl(kd), sl(vd)))
+    out = torch.empty_like(out_ref)
+    streams = [torch.cuda.current_stream(), torch.cuda.Stream()]
+    start, join = torch.cuda.Event(), torch.cuda.Event()
+
+    def layer():
+        start.record(streams[0])
+        streams[1].wait_event(start)
+        for g, (pg, att, qg, kg, vg) in enumerate(groups):
+            st = streams[g % 2]
+            with torch.cuda.stream(st):
+                att(qg, kg, vg, out[:, bounds[g]:bounds[g + 1]], stream=st.cuda_stream)
+        join.record(streams[1])
+        streams[0].wait_event(join)
+
+    for _ in range(3):
+        layer()
+    torch.cuda.synchronize()
+    V.veda_sync_status()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    n = max(3, args.steps // 2)
+    e0.record(streams[0])
+    for _ in range(n):
+        layer()
+    e1.record(streams[0])
+    torch.cuda.synchronize()
+    V.veda_sync_status()
+    return {"groups": G, "streams": 2, "ms_per_layer": e0.elapsed_time(e1) / n, "steps": n,
+            "output_identical": bool(torch.equal(out, out_ref))}
+
+
 def backward_measure(V, w, p, att, qd, kd, vd, args, flops, rank, dev):
     """The attention backward (dQ, dK, dV over the selected tiles) after the
     layer's forward, timed over args.bwd_steps calls with CUDA events.  Its
@@ -610,6 +661,12 @@ def run_ours(args, world, rank, local):
     useful = useful_flops(w, att.idx.cpu().numpy())
     tmap = tile_map_measure(V, w, p, qd, kd, args, rank, att) if args.map else None
     bwd = backward_measure(V, w, p, att, qd, kd, vd, args, flops, rank, dev) if args.bwd else None
+    overlap = None
+    if args.overlap_groups > 1:
+        att(qd, kd, vd, out)
+        overlap = overlap_measure(V, w, qd, kd, vd, mlp, out, args, dev)
+        if "ms_per_layer" in overlap:
+            overlap["one_stream_ms_per_layer"] = ms_step
     if bwd is not None and "ms" in bwd:
         bwd["ratio_to_forward_attention"] = bwd["ms"] / attn_ms
     res = {"metric": METRIC, "value": weak_scaling_value(flops, ms_step, world), "unit": "TFLOP/s",
@@ -628,6 +685,8 @@ def run_ours(args, world, rank, local):
         res["sweep"] = sweep_measure(V, args, dev)
     if bwd is not None:
         res["backward"] = bwd
+    if overlap is not None:
+        res["overlap_prototype"] = overlap
     return res, (w, p, ks, flops)
 
 
@@ -706,6 +765,8 @@ def main():
     ap.add_argument("--bwd-steps", type=int, default=5)
     ap.add_argument("--attn-sustain", type=float, default=0.0,
                     help="also run the attention kernel back to back for this many seconds, sampling clock and power")
+    ap.add_argument("--overlap-groups", type=int, default=0,
+                    help="also time the layer as G head groups on two streams (selection beside attention)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the token sweep record (N = 1 only)")
     ap.add_argument("--sweep-steps", type=int, default=5)
