@@ -110,6 +110,25 @@ def test_workspace_sizes(V):
         V.veda_score_topk_workspace(p, 3)
 
 
+def test_score_workspace_holds_the_score_matrix_for_long_rows(V):
+    """Rows of more than 512 tiles score through the fp32 score matrix in the
+    workspace (e <= 64); shorter rows, and e = 128, keep their scores in shared
+    memory and need only the estimator features."""
+    r256 = lambda x: (x + 255) // 256 * 256
+    def phi(p, e):
+        return r256(4 * 2 * p.B * p.heads * p.nt_max * e)
+    long = V.Problem(1, 4, 128, 128, (21, 45, 80), [(2, 8, 8), (8, 4, 4), (1, 8, 16), (4, 4, 8)])
+    assert long.nt_max == 720
+    pad = (long.nt_max + 3) // 4 * 4
+    for e in (16, 32, 64):
+        assert V.veda_score_topk_workspace(long, e) == phi(long, e) + r256(4 * long.B * long.heads * long.nt_max * pad)
+    assert V.veda_score_topk_workspace(long, 128) == phi(long, 128)
+    short = V.Problem(2, 3, 128, 128, (21, 30, 52), [(2, 8, 8), (8, 4, 4), (1, 8, 16)])
+    assert short.nt_max <= 512
+    for e in (16, 32, 64, 128):
+        assert V.veda_score_topk_workspace(short, e) == phi(short, e)
+
+
 def test_attention_config_query(V):
     """Ring depths and shared memory of the attention launch, computed on the host."""
     p = V.Problem(1, 2, 128, 128, (21, 45, 80), [(2, 8, 8), (8, 4, 4)])
