@@ -94,8 +94,13 @@ class Clocks:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    # Bits of clocks_event_reasons.active (NVML's clock event reasons).
+    ACTIVE_BITS = ((0x1, "gpu_idle"), (0x2, "applications_clocks_setting"), (0x4, "sw_power_cap"),
+                   (0x8, "hw_slowdown"), (0x10, "sync_boost"), (0x20, "sw_thermal_slowdown"),
+                   (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown"),
+                   (0x100, "display_clock_setting"))
 
-    def __init__(self, device_index: int, interval_ms: int = 50):
+    def __init__(self, device_index: int, interval_ms: int = 20):
         self.dev = device_index
         self.interval_ms = interval_ms
         self.proc = None
@@ -117,7 +122,8 @@ class Clocks:
 
     @staticmethod
     def parse(lines):
-        """Rows of (host time or None, sm MHz, max MHz, power W, set of active reasons)."""
+        """Rows of (host time or None, sm MHz, max MHz, power W, set of active
+        named reasons, set of every reason in the active bitmask)."""
         import datetime
         out = []
         for ln in lines:
@@ -133,7 +139,12 @@ class Clocks:
                 except ValueError:
                     pw = None
                 reasons = {n for n, v in zip(Clocks.REASONS, r[6:10]) if v.lower() == "active"}
-                out.append((ts, sm, mx, pw, reasons))
+                try:
+                    mask = int(r[5], 16)
+                except ValueError:
+                    mask = 0
+                active = {n for b, n in Clocks.ACTIVE_BITS if mask & b}
+                out.append((ts, sm, mx, pw, reasons, active))
             except (ValueError, IndexError):
                 continue
         return out
@@ -153,11 +164,14 @@ class Clocks:
                 inside = after[:1] if after else rows[-1:]
         sm = [r[1] for r in inside]
         pw = [r[3] for r in inside if r[3] is not None]
-        reasons = set()
+        reasons, active = set(), set()
         for r in inside:
             reasons |= r[4]
+            active |= r[5]
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(r[2] for r in rows), "reasons": sorted(reasons),
-                "samples": len(inside), "power_w": float(np.median(pw)) if pw else None,
+                "reasons_active": sorted(active), "samples": len(inside),
+                "sm_mhz_samples": [float(x) for x in sm][:64],
+                "power_w": float(np.median(pw)) if pw else None,
                 "window": "timed region" if t0 is not None else "whole run"}
 
     def stop(self):
@@ -183,9 +197,13 @@ def choose_peak(peaks, clk, peak_src):
     median SM clock below its maximum; then the sustained figure (a GEMM run
     for seconds at the power cap) applies.  Returns (peak, basis)."""
     if clk is not None and clk.get("sm_mhz") and clk.get("sm_max_mhz"):
+        active = clk.get("reasons_active", [])
         basis = (f"median SM clock {clk['sm_mhz']:.0f} of {clk['sm_max_mhz']:.0f} MHz over "
-                 f"{clk['samples']} sample(s) in the {clk.get('window', 'run')}, reasons {clk['reasons']}")
-        held_down = bool(clk["reasons"]) and clk["sm_mhz"] < 0.97 * clk["sm_max_mhz"]
+                 f"{clk['samples']} sample(s) in the {clk.get('window', 'run')}, reasons {clk['reasons']}"
+                 + (f", active {active}" if active else ""))
+        throttles = set(clk["reasons"]) | (set(active) & {"sw_power_cap", "hw_power_brake_slowdown", "hw_slowdown",
+                                                           "sw_thermal_slowdown", "hw_thermal_slowdown"})
+        held_down = bool(throttles) and clk["sm_mhz"] < 0.97 * clk["sm_max_mhz"]
         if not held_down:
             return peaks["bf16_tflops"], f"{peak_src} bf16 burst: {basis}"
         return peaks["bf16_tflops_sustained"], f"{peak_src} bf16 sustained (power-capped GEMM): {basis}"

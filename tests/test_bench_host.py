@@ -80,8 +80,28 @@ def test_max_over_ranks_on_two_gloo_ranks():
     assert bench.weak_scaling_value(7.8e12, 15.0, 2) == pytest.approx(2 * 7.8e12 / 15e-3 / 1e12)
 
 
-def _smi_line(ts, sm, mx=1965, pw=500.0, cap="Not Active"):
-    return (f"{ts}, 0, {sm}, {mx}, {pw}, 0x0000000000000000, Not Active, Not Active, Not Active, {cap}")
+def _smi_line(ts, sm, mx=1965, pw=500.0, cap="Not Active", mask="0x0000000000000000"):
+    return (f"{ts}, 0, {sm}, {mx}, {pw}, {mask}, Not Active, Not Active, Not Active, {cap}")
+
+
+def test_clock_active_mask_is_decoded():
+    """Every bit of clocks_event_reasons.active is named in the record, and a
+    hardware power brake holding the clock down selects the sustained peak
+    like the software power cap does."""
+    lines = [_smi_line("2026/12/02 12:00:00.000", 1600, mask="0x0000000000000080"),
+             _smi_line("2026/12/02 12:00:00.020", 1610, mask="0x0000000000000084", cap="Active"),
+             _smi_line("2026/12/02 12:00:00.040", 1620, mask="0x0000000000000001")]
+    clk = bench.Clocks.summarize(bench.Clocks.parse(lines))
+    assert clk["reasons"] == ["sw_power_cap"]
+    assert clk["reasons_active"] == ["gpu_idle", "hw_power_brake_slowdown", "sw_power_cap"]
+    assert clk["sm_mhz_samples"] == [1600.0, 1610.0, 1620.0]
+    peaks = {"bf16_tflops": 1674.3, "bf16_tflops_sustained": 1409.4, "hbm_gbs": 6541.8}
+    brake_only = {"sm_mhz": 1600.0, "sm_max_mhz": 1965.0, "reasons": [], "reasons_active": ["hw_power_brake_slowdown"],
+                  "samples": 3, "window": "timed region"}
+    peak, basis = bench.choose_peak(peaks, brake_only, "measured")
+    assert peak == 1409.4 and "hw_power_brake_slowdown" in basis
+    idle_only = dict(brake_only, reasons_active=["gpu_idle"])
+    assert bench.choose_peak(peaks, idle_only, "measured")[0] == 1674.3
 
 
 def test_clock_summary_keeps_only_the_timed_region():
