@@ -577,6 +577,9 @@ def run_ours(args, world, rank, local):
         V.veda_tile_score_topk(p, att.desc_q, att.desc_k, att.mlp_q, att.mlp_k, att.keep, att.idx, None,
                                att.workspace)
 
+    # Rows of more than 512 tiles (e <= 64) score through the score matrix in
+    # the workspace: the score GEMM is one more launch.
+    sel_extra = 1 if (w.e <= 64 and p.nt_max > 512) else 0
     if args.layout == "tile":
         stages = [("permute_tripool_qk", lambda: (V.veda_tile_permute_tripool(p, qd, att.qp, att.desc_q),
                                                   V.veda_tile_permute_tripool(p, kd, att.kp, att.desc_k))),
@@ -584,14 +587,15 @@ def run_ours(args, world, rank, local):
                   ("score_topk", score),
                   ("attention", lambda: V.veda_tile_sparse_attn(p, att.qp, att.kp, att.vp, att.idx, att.op)),
                   ("unpermute", lambda: V.veda_tile_unpermute(p, att.op, out))]
-        launches_per_step = 7       # 2 permute+TripPool, permute, estimator, top-k, attention, unpermute
+        launches_per_step = 7 + sel_extra   # 2 permute+TripPool, permute, estimator, top-k, attention, unpermute
     else:
         stages = [("tripool_qk", lambda: (V.veda_tripool_grid(p, qd, att.desc_q),
                                           V.veda_tripool_grid(p, kd, att.desc_k))),
                   ("score_topk", score),
                   ("attention", lambda: V.veda_tile_sparse_attn_grid(p, qd, kd, vd, att.idx, out))]
         n_tilings = len(set(w.tilings))
-        launches_per_step = 4 + (n_tilings + 7) // 8   # 2 TripPool, estimator, top-k, attention per 8 tilings
+        # 2 TripPool, estimator, top-k (+ the score GEMM), attention per 8 tilings
+        launches_per_step = 4 + sel_extra + (n_tilings + 7) // 8
 
     def step(ev=None):
         if ev is None:
