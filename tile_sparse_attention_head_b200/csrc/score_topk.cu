@@ -799,8 +799,9 @@ __global__ void __launch_bounds__(kTrWarps * 32)
 
 // Bytes of the score matrix in the workspace, 0 when the fused kernels score:
 // for e = 128, and for rows of up to 512 tiles, where the fused kernel is
-// faster (Wan2.1-1.3B: 0.062 against 0.073 ms for estimator plus selection;
-// Wan2.1-14B, 720 tiles: 0.314 against 0.265 ms).
+// faster.  Estimator plus selection, fused kernel against score matrix:
+// Wan2.1-1.3B (336 tiles) 0.062 against 0.073 ms, Wan2.1-14B (720 tiles)
+// 0.314 against 0.265 ms.
 size_t score_matrix_bytes(const Geometry& G, int e) {
   if (e > 64 || G.ntmax <= 512) return 0;
   return sizeof(float) * (size_t)G.B * G.heads * G.ntmax * (size_t)((G.ntmax + 3) & ~3);
